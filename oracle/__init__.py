@@ -1,0 +1,9 @@
+"""CPU oracle for the theta-bundle path (test infrastructure, not the product).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU baseline leg
+may import this package.
+"""
+from .theta_oracle import (  # noqa: F401
+    round_to, band_sizes, band_index, band_mean, row_scale, residual,
+    truncated_svd, reconstruct, frob_error, linear_forward, decompose_family,
+)

@@ -1,0 +1,203 @@
+"""Plain fp64 CPU oracle for the theta-bundle projection path.
+
+TEST INFRASTRUCTURE ONLY. This module is the independent checker for the GPU
+library: only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU
+baseline leg may import it. The product path never calls it, and it shares no
+code with the CUDA implementation (it imports neither torch nor the library).
+
+Every function is the definition from the pages written out with numpy in
+float64, no blocking, no fusion, no reordering beyond what the definition
+states. Inputs arrive as float32 arrays whose values are exact in their
+storage dtype (f32 or bf16); they are upcast exactly to float64. Results that
+the GPU stores in a narrower dtype are rounded once, round-to-nearest-even,
+by ``round_to``.
+
+Sources (page title -- section):
+  * "Banded sharing" -- How layers map to bands: G contiguous bands, as equal
+    as possible, earlier bands take the remainder.
+  * "The theta bundle" -- table of components (W0 [out,in], s [out],
+    U [out,rank], V [in,rank]); the approximation weight ~ diag(s)·W0 + U·Vᵀ;
+    Analytic decomposition (Shared block, Per-row scale, Low-rank residual);
+    reconstruct_weight / relative_frobenius_error.
+  * "Quality" -- Native-equivalent at passthrough (G = num_layers rebuilds the
+    weight exactly); Reconstruction error (relative Frobenius error).
+
+Readings where the pages are silent (each one is listed in the design doc):
+  * G outside [1, num_layers] is rejected.
+  * W0 is the fp64 mean, rounded once to the storage dtype.
+  * s is fitted against the *stored* (rounded) W0, the block the forward uses.
+  * A row whose W0·W0 is zero gets s = 0 (minimum-norm least squares).
+  * relative_frobenius_error = ||A - B||_F / ||A||_F; 0/0 -> 0, x/0 -> inf.
+  * The forward has no bias term; its output dtype is the activations' dtype.
+
+Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
+against closed forms, brute force on tiny inputs, library routines and the
+passthrough invariant. None is "parity unpinned".
+"""
+from __future__ import annotations
+
+import numpy as np
+
+F64 = np.float64
+
+# significand bits and smallest quantum exponent of each storage dtype
+_FORMATS = {"f32": (24, -149), "bf16": (8, -133)}
+_MAX_FINITE_EXP = 128  # both f32 and bf16 overflow at 2**128
+
+
+# ------------------------------------------------------------------ rounding
+def round_to(x, dtype: str) -> np.ndarray:
+    """Round float64 values to the nearest value of ``dtype`` (ties to even).
+
+    A value with binary exponent e (2**(e-1) <= |x| < 2**e) has quantum
+    2**(e - p) in a format with p significand bits; subnormals share the
+    smallest quantum. np.rint rounds half to even.
+    """
+    a = np.asarray(x, dtype=F64)
+    if dtype == "f64":
+        return a.copy()
+    p, qmin = _FORMATS[dtype]
+    _, e = np.frexp(a)
+    q = np.maximum(e - p, qmin)
+    y = np.ldexp(np.rint(np.ldexp(a, -q)), q)
+    over = np.abs(y) >= 2.0 ** _MAX_FINITE_EXP
+    if np.any(over):
+        y = np.where(over, np.copysign(np.inf, a), y)
+    return y
+
+
+# ------------------------------------------------------------- banded sharing
+def band_sizes(num_layers: int, G: int) -> list[int]:
+    """Sizes of the G contiguous bands ("Banded sharing" -- How layers map to bands).
+
+    As equal as possible: every band holds num_layers // G layers, and the
+    num_layers % G leftover layers go one each to the earliest bands.
+    """
+    if not (isinstance(num_layers, int) and isinstance(G, int)):
+        raise TypeError("num_layers and G must be int")
+    if num_layers < 1 or G < 1 or G > num_layers:
+        raise ValueError(f"need 1 <= G <= num_layers, got G={G}, num_layers={num_layers}")
+    base, extra = divmod(num_layers, G)
+    return [base + 1 if b < extra else base for b in range(G)]
+
+
+def band_index(num_layers: int, G: int):
+    """(band_of_layer[num_layers], band_start[G + 1]) as int32 arrays."""
+    sizes = band_sizes(num_layers, G)
+    start = np.zeros(G + 1, dtype=np.int32)
+    start[1:] = np.cumsum(sizes)
+    band_of_layer = np.empty(num_layers, dtype=np.int32)
+    for b in range(G):
+        band_of_layer[start[b]:start[b + 1]] = b
+    return band_of_layer, start
+
+
+# ---------------------------------------------------------- decomposition
+def band_mean(weights, G: int, out_dtype: str = "f64") -> np.ndarray:
+    """W0[b] = mean of the band's layer weights ("The theta bundle" -- Shared block).
+
+    weights: [L, O, I]. Returns [G, O, I] rounded to ``out_dtype``.
+    """
+    w = np.asarray(weights, dtype=F64)
+    _, start = band_index(w.shape[0], G)
+    out = np.empty((G,) + w.shape[1:], dtype=F64)
+    for b in range(G):
+        out[b] = w[start[b]:start[b + 1]].mean(axis=0)
+    return round_to(out, out_dtype)
+
+
+def row_scale(weight, W0) -> np.ndarray:
+    """s_r = (w_r · W0_r) / (W0_r · W0_r) per output row r
+    ("The theta bundle" -- Per-row scale). Rows with W0_r = 0 get s_r = 0.
+    """
+    w = np.asarray(weight, dtype=F64)
+    w0 = np.asarray(W0, dtype=F64)
+    num = np.einsum("oi,oi->o", w, w0)
+    den = np.einsum("oi,oi->o", w0, w0)
+    s = np.zeros_like(num)
+    nz = den != 0
+    s[nz] = num[nz] / den[nz]
+    return s
+
+
+def residual(weight, W0, s, out_dtype: str = "f64") -> np.ndarray:
+    """weight - diag(s)·W0 ("The theta bundle" -- Low-rank residual)."""
+    w = np.asarray(weight, dtype=F64)
+    w0 = np.asarray(W0, dtype=F64)
+    sc = np.asarray(s, dtype=F64)
+    return round_to(w - sc[:, None] * w0, out_dtype)
+
+
+def truncated_svd(R, rank: int):
+    """Rank-r factors of the residual with U absorbing the singular values
+    ("The theta bundle" -- Low-rank residual). Full LAPACK SVD, for small
+    matrices only. Returns (U [O, r], V [I, r]) with U·Vᵀ ~ R.
+    """
+    Rm = np.asarray(R, dtype=F64)
+    if rank == 0:
+        return np.zeros((Rm.shape[0], 0)), np.zeros((Rm.shape[1], 0))
+    Uf, sig, Vt = np.linalg.svd(Rm, full_matrices=False)
+    return Uf[:, :rank] * sig[:rank], Vt[:rank].T.copy()
+
+
+def reconstruct(s, W0, U, V, out_dtype: str = "f64") -> np.ndarray:
+    """reconstruct_weight(s, W0, U, V) = diag(s)·W0 + U·Vᵀ
+    ("The theta bundle" -- the approximation formula and Key layout)."""
+    sc = np.asarray(s, dtype=F64)
+    w0 = np.asarray(W0, dtype=F64)
+    Um = np.asarray(U, dtype=F64).reshape(w0.shape[0], -1)
+    Vm = np.asarray(V, dtype=F64).reshape(w0.shape[1], -1)
+    return round_to(sc[:, None] * w0 + Um @ Vm.T, out_dtype)
+
+
+def frob_error(original, reconstructed) -> float:
+    """relative_frobenius_error = ||A - B||_F / ||A||_F ("Quality" --
+    Reconstruction error). 0 when both norms are 0, +inf when only ||A|| is."""
+    A = np.asarray(original, dtype=F64)
+    B = np.asarray(reconstructed, dtype=F64)
+    num = np.sqrt(np.sum((A - B) ** 2))
+    den = np.sqrt(np.sum(A ** 2))
+    if den == 0.0:
+        return 0.0 if num == 0.0 else float("inf")
+    return float(num / den)
+
+
+# ----------------------------------------------------------------- forward
+def linear_forward(X, W0, s, U, V, out_dtype: str = "f64") -> np.ndarray:
+    """Y = X·(diag(s)·W0 + U·Vᵀ)ᵀ = s ⊙ (X·W0ᵀ) + (X·V)·Uᵀ.
+
+    The projection applies the rebuilt weight of "The theta bundle" to the
+    activations without forming it; X [M, I] -> Y [M, O].
+    """
+    Xm = np.asarray(X, dtype=F64)
+    w0 = np.asarray(W0, dtype=F64)
+    sc = np.asarray(s, dtype=F64)
+    Um = np.asarray(U, dtype=F64).reshape(w0.shape[0], -1)
+    Vm = np.asarray(V, dtype=F64).reshape(w0.shape[1], -1)
+    Y = sc[None, :] * (Xm @ w0.T) + (Xm @ Vm) @ Um.T
+    return round_to(Y, out_dtype)
+
+
+# -------------------------------------------------------- whole decomposition
+def decompose_family(weights, G: int, rank: int, dtype: str = "f64"):
+    """Analytic decomposition of one projection family, in the pages' order:
+    band means, then per layer the row scale against its band's stored W0, the
+    residual, and its rank-r truncated SVD. Returns a dict with W0 [G,O,I],
+    s [L,O], R [L,O,I], U [L,O,r], V [L,I,r], band_of_layer [L].
+    """
+    w = np.asarray(weights, dtype=F64)
+    L = w.shape[0]
+    band_of_layer, _ = band_index(L, G)
+    W0 = band_mean(w, G, dtype)
+    s = np.empty((L, w.shape[1]))
+    R = np.empty_like(w)
+    Us, Vs = [], []
+    for layer in range(L):
+        w0 = W0[band_of_layer[layer]]
+        s[layer] = row_scale(w[layer], w0)
+        R[layer] = residual(w[layer], w0, s[layer], dtype)
+        U, V = truncated_svd(R[layer], rank)
+        Us.append(U)
+        Vs.append(V)
+    return {"W0": W0, "s": s, "R": R, "U": np.stack(Us), "V": np.stack(Vs),
+            "band_of_layer": band_of_layer}
