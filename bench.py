@@ -1,0 +1,575 @@
+#!/usr/bin/env python
+"""Throughput of the theta-bundle hot path on B200.
+
+One step is one pass of every stage of the path over one synthetic workload,
+Gemma-3-1B-shaped: 26 layers, the seven projection families (q [1024,1152],
+k/v [256,1152], o [1152,1024], gate/up [6912,1152], down [1152,6912]), bf16
+weights drawn as a common N(0,0.02) base plus per-layer N(0,0.005) noise,
+rank-32 factors U, V ~ N(0,0.01), activations X ~ N(0,1). For each of
+G = 26 (passthrough) and G = 1 the step runs, per family:
+
+  prelude      band means W0, row scales s and residuals R  (theta_decompose_prelude)
+  reconstruct  diag(s).W0 + U.V^T for every layer           (theta_reconstruct)
+  frob         ||W - W_rec||_F / ||W||_F for every layer     (theta_frob_error)
+  forward      s*(X.W0^T) + (X.V).U^T for every layer at M = 1, 16, 256
+                                                             (theta_linear_forward)
+
+Throughput is algorithmic bytes per second: the bytes each call must move at
+minimum (inputs read once, outputs written once; W0 counted once per forward
+call), summed over the step, divided by the device time of the step. Each
+stage is captured as a CUDA graph; the step replays them back to back with
+CUDA events between stages. The step touches > 10 GB, far more than the 126 MB
+L2, so no explicit flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun each rank runs the whole workload on its own GPU (independent
+problems, weak scaling); rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synthetic as syn  # noqa: E402
+
+METRIC = "theta-forward TFLOP/s (prefill) & GB/s (decode) vs B200 roofline; decompose GB/s"
+WORKLOAD = "gemma3-1b-shaped theta path: 26 layers x 7 families, bf16, G in {26,1}, rank 32, M in {1,16,256}"
+MODEL = syn.GEMMA3_1B
+RANK = 32
+M_VALUES = (1, 16, 256)
+G_VALUES = (26, 1)
+BF16 = 2  # bytes
+
+
+# --------------------------------------------------------------- accounting
+def bytes_band_mean(L, G, O, I, b=BF16):
+    return L * O * I * b + G * O * I * b
+
+
+def bytes_rowscale_residual(L, G, O, I, b=BF16):
+    # read every W once and each band's W0 once; write s (fp32) and R
+    return L * O * I * b + G * O * I * b + 4 * L * O + L * O * I * b
+
+
+def bytes_reconstruct(O, I, r, b=BF16):
+    return O * I * b + 4 * O + r * (O + I) * b + O * I * b
+
+
+def bytes_frob(O, I, b=BF16):
+    return 2 * O * I * b
+
+
+def bytes_forward(M, O, I, r, b=BF16):
+    return O * I * b + 4 * O + r * (O + I) * b + M * I * b + M * O * b
+
+
+def flops_forward(M, O, I, r):
+    return 2 * M * (O * I + r * (I + O))
+
+
+def step_accounting(model=MODEL, r=RANK, m_values=M_VALUES, g_values=G_VALUES):
+    """Per-stage algorithmic bytes / flops / kernel launches of one step."""
+    L = model.num_layers
+    stages = []
+    for G in g_values:
+        pre = rec = fro = 0
+        fwd = {m: [0, 0] for m in m_values}
+        for fam, (O, I) in model.shapes.items():
+            pre += bytes_band_mean(L, G, O, I) + bytes_rowscale_residual(L, G, O, I)
+            rec += L * bytes_reconstruct(O, I, r)
+            fro += L * bytes_frob(O, I)
+            for m in m_values:
+                fwd[m][0] += L * bytes_forward(m, O, I, r)
+                fwd[m][1] += L * flops_forward(m, O, I, r)
+        nf = len(model.shapes)
+        stages.append(dict(name=f"prelude_G{G}", kind="prelude", bytes=pre, flops=0, launches=nf * G * 2))
+        stages.append(dict(name=f"reconstruct_G{G}", kind="reconstruct", bytes=rec, flops=0, launches=nf * L))
+        stages.append(dict(name=f"frob_G{G}", kind="frob", bytes=fro, flops=0, launches=nf * L * 2))
+        for m in m_values:
+            stages.append(dict(name=f"forward_m{m}_G{G}", kind=f"forward_m{m}", bytes=fwd[m][0],
+                               flops=fwd[m][1], launches=nf * L * (2 if r > 0 else 1)))
+    return stages
+
+
+# --------------------------------------------------------------- environment
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": p["hbm_gbs"], "bf16_tflops": p["bf16_tflops"],
+                "bf16_tflops_sustained": p.get("bf16_tflops_sustained", p["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank number over all ranks (identity for one process)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def result_line(*, value, unit, n_gpus, steps, warmup, ms_per_step, extra):
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": n_gpus, "steps": steps, "warmup": warmup,
+            "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (seeded; weights, factors and activations drawn on the device)"}
+    line.update(extra)
+    return line
+
+
+# --------------------------------------------------------------- workload
+class Workload:
+    """All device tensors of one step, and the stage call lists."""
+
+    def __init__(self, theta, torch, seed=0, model=MODEL, r=RANK):
+        self.theta, self.torch = theta, torch
+        self.model, self.r, self.L = model, r, model.num_layers
+        dev = "cuda"
+        bf = torch.bfloat16
+        L = self.L
+        self.W, self.W0, self.s, self.R, self.rec, self.U, self.V = {}, {}, {}, {}, {}, {}, {}
+        for fam, (O, I) in model.shapes.items():
+            self.W[fam] = syn.device_family_weights(L, O, I, seed=seed, family=fam, dtype="bf16")
+            self.W0[fam] = [torch.empty(O, I, dtype=bf, device=dev) for _ in range(max(G_VALUES))]
+            self.s[fam] = [torch.empty(O, dtype=torch.float32, device=dev) for _ in range(L)]
+            self.R[fam] = [torch.empty(O, I, dtype=bf, device=dev) for _ in range(L)]
+            self.rec[fam] = [torch.empty(O, I, dtype=bf, device=dev) for _ in range(L)]
+            self.U[fam] = [syn.device_normal((O, r), 0.01, seed, "U", fam, l) for l in range(L)]
+            self.V[fam] = [syn.device_normal((I, r), 0.01, seed, "V", fam, l) for l in range(L)]
+        in_dims = sorted({I for (_, I) in model.shapes.values()})
+        self.X = {(m, I): syn.device_normal((m, I), 1.0, seed, "X", m, I) for m in M_VALUES for I in in_dims}
+        self.Y = {(m, fam, l): torch.empty(m, O, dtype=bf, device=dev)
+                  for m in M_VALUES for fam, (O, _) in model.shapes.items() for l in range(L)}
+        self.frob_out = torch.zeros(len(G_VALUES), len(model.shapes), L, dtype=torch.float64, device=dev)
+        fb = theta.theta_workspace_size(theta.THETA_OP_FROB_ERROR, 1, 1, 1, 0, theta.THETA_BF16)
+        self.frob_ws = torch.empty(fb, dtype=torch.uint8, device=dev)
+        wb = max(theta.theta_workspace_size(theta.THETA_OP_LINEAR_FORWARD, m, O, I, r, theta.THETA_BF16)
+                 for m in M_VALUES for (O, I) in model.shapes.values())
+        self.fwd_ws = torch.empty(max(wb, 256), dtype=torch.uint8, device=dev)
+        self.bands = {G: theta.theta_band_index(L, G)[0] for G in G_VALUES}
+
+    # stage bodies ------------------------------------------------------
+    def prelude(self, G):
+        t = self.theta
+        for fam in self.model.shapes:
+            t.theta_decompose_prelude(self.W[fam], G, self.W0[fam][:G], self.s[fam], self.R[fam])
+
+    def reconstruct(self, G):
+        t = self.theta
+        for fam in self.model.shapes:
+            band = self.bands[G]
+            for l in range(self.L):
+                t.theta_reconstruct(self.s[fam][l], self.W0[fam][band[l]], self.U[fam][l], self.V[fam][l],
+                                    self.rec[fam][l])
+
+    def frob(self, G):
+        t = self.theta
+        gi = G_VALUES.index(G)
+        for fi, fam in enumerate(self.model.shapes):
+            for l in range(self.L):
+                t.theta_frob_error(self.W[fam][l], self.rec[fam][l], self.frob_out[gi, fi, l:l + 1],
+                                   self.frob_ws)
+
+    def forward(self, G, m):
+        t = self.theta
+        band = self.bands[G]
+        for fam, (O, I) in self.model.shapes.items():
+            X = self.X[(m, I)]
+            for l in range(self.L):
+                t.theta_linear_forward(X, self.W0[fam][band[l]], self.s[fam][l], self.U[fam][l], self.V[fam][l],
+                                       self.Y[(m, fam, l)], self.fwd_ws)
+
+    def stage_fns(self):
+        fns = []
+        for G in G_VALUES:
+            fns.append(lambda G=G: self.prelude(G))
+            fns.append(lambda G=G: self.reconstruct(G))
+            fns.append(lambda G=G: self.frob(G))
+            for m in M_VALUES:
+                fns.append(lambda G=G, m=m: self.forward(G, m))
+        return fns
+
+    # host side of the end-to-end run -----------------------------------
+    def input_tensors(self):
+        ins = []
+        for fam in self.model.shapes:
+            ins += self.W[fam] + self.U[fam] + self.V[fam]
+        ins += list(self.X.values())
+        return ins
+
+    def output_tensors(self):
+        return [self.frob_out] + list(self.Y.values()) + [s for fam in self.model.shapes for s in self.s[fam]]
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "linear_theta_forward_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kind):
+    """DRAM bytes per launch of a stage's main kernel from a committed ncu
+    capture, or None when the kernels changed since it was taken."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f)
+    entry = rec.get(kind)
+    if not entry or entry.get("source_hash") != kernel_source_hash():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------- CPU oracle
+def oracle_sample_step(rows=64, seed=0, model=MODEL, r=RANK):
+    """One bounded sample of the step on the host CPU with the fp64 oracle:
+    the first `rows` output rows of every family, all layers, both G values.
+    Inputs are drawn before the clock starts. Returns (algorithmic bytes of
+    the sample, seconds)."""
+    import oracle
+    L = model.num_layers
+    inputs = {}
+    for fam, (O, I) in model.shapes.items():
+        n = min(rows, O)
+        w = syn.host_family_weights(L, n, I, seed=seed, family=f"cpu-{fam}", dtype="bf16")
+        U = [syn.host_normal((n, r), 0.01, seed, "U", fam, l, dtype="bf16") for l in range(L)]
+        V = [syn.host_normal((I, r), 0.01, seed, "V", fam, l, dtype="bf16") for l in range(L)]
+        X = {m: syn.host_activations(m, I, seed=seed, tag=f"cpu-{m}", dtype="bf16") for m in M_VALUES}
+        inputs[fam] = (n, I, w, U, V, X)
+    total_bytes = 0
+    t0 = time.perf_counter()
+    for fam, (n, I, w, U, V, X) in inputs.items():
+        for G in G_VALUES:
+            band, _ = oracle.band_index(L, G)
+            W0 = oracle.band_mean(w, G, "bf16")
+            for l in range(L):
+                w0 = W0[band[l]]
+                s = oracle.row_scale(w[l], w0)
+                oracle.residual(w[l], w0, s, "bf16")
+                s32 = oracle.round_to(s, "f32")
+                rec = oracle.reconstruct(s32, w0, U[l], V[l], "bf16")
+                oracle.frob_error(w[l], rec)
+                for m in M_VALUES:
+                    oracle.linear_forward(X[m], w0, s32, U[l], V[l], "bf16")
+            total_bytes += bytes_band_mean(L, G, n, I) + bytes_rowscale_residual(L, G, n, I)
+            total_bytes += L * (bytes_reconstruct(n, I, r) + bytes_frob(n, I))
+            total_bytes += L * sum(bytes_forward(m, n, I, r) for m in M_VALUES)
+    return total_bytes, time.perf_counter() - t0
+
+
+def cpu_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = max((d.get("num_threads", 1) for d in info), default=1)
+        return int(n)
+    except Exception:
+        return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(target_s=12.0, rows=64):
+    np.ones((64, 64)) @ np.ones((64, 64))  # load BLAS so its threads are visible
+    done_bytes, spent, reps = 0, 0.0, 0
+    while spent < target_s and reps < 50:
+        b, s = oracle_sample_step(rows=rows, seed=reps)
+        done_bytes += b
+        spent += s
+        reps += 1
+    return {"value": done_bytes / spent / 1e9, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{reps} x (first {rows} output rows of each of the 7 families, all 26 layers, "
+                      f"G in {{26,1}}, every stage incl. forward at M in {{1,16,256}}); {spent:.1f} s"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: each step is one bounded row sample."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    oracle_sample_step(rows=16)  # warm the imports and BLAS
+    for _ in range(args.warmup):
+        oracle_sample_step(rows=args.ref_rows)
+    times, nbytes = [], 0
+    for i in range(args.steps):
+        b, s = oracle_sample_step(rows=args.ref_rows, seed=i)
+        times.append(s)
+        nbytes = b
+    per_step = sum(times) / len(times)
+    value = nbytes / per_step / 1e9
+    line = result_line(value=value, unit="GB/s", n_gpus=args.gpus, steps=args.steps, warmup=args.warmup,
+                       ms_per_step=per_step * 1e3, extra={
+                           "impl": "reference", "dtype": "f64",
+                           "config": {"workload": WORKLOAD, "sample_rows_per_family": args.ref_rows,
+                                      "l2": "n/a (CPU)"},
+                           "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+                                            "sample": f"first {args.ref_rows} output rows of each family per step"},
+                           "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+                       })
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------- GPU arm
+def run_gpu(args):
+    import torch
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    import linear_theta_forward_b200 as theta
+
+    peaks = measured_peaks()
+    wl = Workload(theta, torch, seed=rank)
+    stages = step_accounting()
+    fns = wl.stage_fns()
+    assert len(fns) == len(stages)
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+
+    # one eager pass (initialises the library), then capture every stage
+    with torch.cuda.stream(stream):
+        for fn in fns:
+            fn()
+    theta.theta_device_status(stream)
+    graphs = []
+    if not args.no_graph:
+        for fn in fns:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+            graphs.append(g)
+    run = [g.replay for g in graphs] if graphs else fns
+
+    def one_step(events=None):
+        with torch.cuda.stream(stream):
+            for i, f in enumerate(run):
+                if events is not None:
+                    events[i].record(stream)
+                f()
+            if events is not None:
+                events[-1].record(stream)
+
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+    theta.theta_device_status(stream)
+
+    n_st = len(stages)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_st + 1)] for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        start = torch.cuda.Event(enable_timing=True)
+        stop = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for k in range(args.steps):
+            one_step(ev[k])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    theta.theta_device_status(stream)
+    total_ms = max_over_ranks(start.elapsed_time(stop), world, device="cuda")
+    stage_ms = [sum(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(args.steps)) / args.steps
+                for i in range(n_st)]
+
+    step_bytes = sum(s["bytes"] for s in stages)
+    ms_per_step = total_ms / args.steps
+    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+    launches = sum(s["launches"] for s in stages) * args.steps
+
+    # per-kind aggregates; the dominant kind gives the roofline entry
+    kinds = {}
+    for st, ms in zip(stages, stage_ms):
+        k = kinds.setdefault(st["kind"], {"ms": 0.0, "bytes": 0, "flops": 0, "launches": 0})
+        k["ms"] += ms
+        k["bytes"] += st["bytes"]
+        k["flops"] += st["flops"]
+        k["launches"] += st["launches"]
+    parts = {}
+    for name, k in kinds.items():
+        parts[name] = {"ms": round(k["ms"], 4), "GB/s": round(k["bytes"] / (k["ms"] * 1e-3) / 1e9, 1),
+                       "frac_hbm": round(k["bytes"] / (k["ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"], 3)}
+        if k["flops"]:
+            parts[name]["TFLOP/s"] = round(k["flops"] / (k["ms"] * 1e-3) / 1e12, 2)
+    dom_name, dom = max(kinds.items(), key=lambda kv: kv[1]["ms"])
+    per_launch_bytes = dom["bytes"] / dom["launches"]
+    per_launch_s = dom["ms"] * 1e-3 / dom["launches"]
+    achieved = per_launch_bytes / per_launch_s / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": recorded_traffic(dom_name),
+                "kernel": dom_name, "peak_source": peaks["source"],
+                "bytes_per_launch": round(per_launch_bytes), "launches_per_step": dom["launches"]}
+
+    e2e = None
+    if not args.skip_e2e:
+        e2e = run_e2e(torch, theta, wl, run, stream, step_bytes, min(args.steps, args.e2e_steps), world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        cpu = cpu_baseline(target_s=args.cpu_seconds)
+
+    if rank == 0:
+        line = result_line(value=round(value, 2), unit="GB/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
+                           ms_per_step=round(ms_per_step, 4), extra={
+                               "config": {"workload": WORKLOAD, "model": "gemma3-1b-shaped (random init)",
+                                          "layers": MODEL.num_layers, "families": list(MODEL.shapes),
+                                          "G": list(G_VALUES), "rank": RANK, "M": list(M_VALUES),
+                                          "global_batch": max(M_VALUES), "seq_len": 1,
+                                          "parallelism": f"independent replicas x{world}",
+                                          "graphs": not args.no_graph,
+                                          "l2": "inputs larger than L2 (>10 GB touched per step); no flush"},
+                               "parts": parts,
+                               "roofline": roofline,
+                               "cpu_baseline": cpu,
+                               "e2e": e2e,
+                               "gpu_launches": launches,
+                               "clocks": clocks.summary(),
+                           })
+        print(json.dumps(line), flush=True)
+    for g in graphs:
+        del g
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def run_e2e(torch, theta, wl, run, stream, step_bytes, steps, world):
+    """The same step through the public API with HOST buffers: every step copies
+    its inputs from pinned host memory, runs, and reads its results back."""
+    ins = wl.input_tensors()
+    outs = wl.output_tensors()
+    h_in = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in ins]
+    for h, t in zip(h_in, ins):
+        h.copy_(t)
+    h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in ins)
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    stop = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for _ in range(steps):
+            for h, t in zip(h_in, ins):
+                t.copy_(h, non_blocking=True)
+            for f in run:
+                f()
+            for h, t in zip(h_out, outs):
+                h.copy_(t, non_blocking=True)
+        stop.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(start.elapsed_time(stop), world, device="cuda") / steps
+    return {"value": round(world * step_bytes / (ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3), "steps": steps}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-rows", type=int, default=32)
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "native":
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,211 @@
+/*
+ * libtheta -- theta-bundle projections on NVIDIA B200 (sm_100a).
+ *
+ * A decoder projection weight W [out_dim O, in_dim I] is represented by a
+ * theta bundle ("The theta bundle" -- component table and approximation
+ * formula):
+ *
+ *     W  ~  diag(s) . W0[band] + U . V^T
+ *
+ *   W0 [O, I]  shared block: the mean of the family's weights over a
+ *              contiguous band of layers ("Banded sharing");
+ *   s  [O]     per-output-row least-squares scale against W0 (fp32 always);
+ *   U  [O, r]  left factor of the rank-r residual (absorbs the singular values);
+ *   V  [I, r]  right factor (stored [in_dim, rank], not transposed).
+ *
+ * Conventions for every call
+ *   - Matrices are dense, row-major, with no padding: row pitch = columns.
+ *     X [M, I], W0 [O, I], U [O, r], V [I, r], Y [M, O].
+ *   - Element type: THETA_F32 (fp32 everywhere) or THETA_BF16 (bf16 storage,
+ *     fp32 arithmetic and accumulation). s is always fp32.
+ *   - "device" pointers point to memory of the current CUDA device; "host"
+ *     pointers to host memory. The caller owns every buffer; the library keeps
+ *     no pointer after a call returns and allocates no device memory.
+ *   - Calls taking a stream are asynchronous: they validate arguments on the
+ *     host, enqueue kernels on `stream` (a cudaStream_t; NULL means the legacy
+ *     default stream) and return. Errors found on the host are returned before
+ *     anything is enqueued; nothing is written in that case.
+ *   - THETA_BF16 calls use the Tensor Memory Accelerator and need 16-byte
+ *     aligned base pointers and row pitches that are multiples of 16 bytes
+ *     (I, O and r multiples of 8); otherwise they return THETA_ERR_ALIGNMENT.
+ *   - Kernels bound every wait they make. A wait that runs out records a flag
+ *     on the device and the kernel returns early; theta_device_status() reports
+ *     it as THETA_ERR_TIMEOUT.
+ *   - theta_last_error() gives a message for the last failing call on the
+ *     calling thread.
+ */
+#ifndef THETA_H
+#define THETA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define THETA_VERSION 1
+#define THETA_MAX_LAYERS 256 /* layers per call of the band/prelude entry points */
+
+typedef enum {
+  THETA_OK = 0,
+  THETA_ERR_INVALID_ARG = -1, /* bad size, count, pointer or dtype */
+  THETA_ERR_UNSUPPORTED = -2, /* valid request this build cannot serve */
+  THETA_ERR_ALIGNMENT = -3,   /* TMA alignment rule broken (bf16 paths) */
+  THETA_ERR_CUDA = -4,        /* CUDA runtime/driver error; see theta_last_error */
+  THETA_ERR_TIMEOUT = -5,     /* a bounded device wait ran out */
+  THETA_ERR_WORKSPACE = -6    /* workspace missing or smaller than required */
+} theta_status;
+
+typedef enum { THETA_F32 = 0, THETA_BF16 = 1 } theta_dtype;
+
+typedef enum {
+  THETA_OP_FROB_ERROR = 0,
+  THETA_OP_LINEAR_FORWARD = 1
+} theta_op;
+
+/* Library version (THETA_VERSION of the build). */
+int theta_version(void);
+
+/* Static name of a status code. */
+const char* theta_status_string(int status);
+
+/* Message of the last failing call on this thread ("" if none). The pointer
+ * stays valid until the next libtheta call on the same thread. */
+const char* theta_last_error(void);
+
+/*
+ * theta_band_index -- layer-to-band map ("Banded sharing" -- How layers map
+ * to bands): num_layers layers form G contiguous bands, as equal in size as
+ * possible, the earlier bands taking the remainder. With q = num_layers / G
+ * and m = num_layers % G, band b has q + 1 layers if b < m, else q.
+ *
+ *   band_of_layer  host int32[num_layers], written: band of each layer.
+ *   band_start     host int32[G + 1] or NULL, written: first layer of each
+ *                  band, band_start[G] = num_layers.
+ * Synchronous and host-only (no CUDA call). Returns THETA_ERR_INVALID_ARG
+ * unless 1 <= G <= num_layers and band_of_layer is non-NULL.
+ */
+int theta_band_index(int num_layers, int G, int32_t* band_of_layer, int32_t* band_start);
+
+/*
+ * theta_band_mean -- shared block of one band ("The theta bundle" --
+ * Analytic decomposition, Shared block): W0 = (1/n) sum_l W_l over the n
+ * given layers. Accumulates in fp32 in layer order, divides once by n and
+ * rounds once to dt.
+ *
+ *   weights  host array of n device pointers, each [O, I] of dt.
+ *   W0       device [O, I] of dt, written.
+ * 1 <= n <= THETA_MAX_LAYERS; O, I >= 1.
+ */
+int theta_band_mean(const void* const* weights, int n, int64_t O, int64_t I, theta_dtype dt,
+                    void* W0, void* stream);
+
+/*
+ * theta_row_scale -- per-row least-squares scale ("The theta bundle" --
+ * Per-row scale): s[o] = <W[o,:], W0[o,:]> / <W0[o,:], W0[o,:]>, both dot
+ * products in fp32 with the same summation order (so W == W0 gives s == 1
+ * exactly). A row with <W0,W0> == 0 gets s = 0.
+ *
+ *   weight device [O, I] of dt;  W0 device [O, I] of dt;  s device fp32 [O], written.
+ */
+int theta_row_scale(const void* weight, const void* W0, int64_t O, int64_t I, theta_dtype dt,
+                    float* s, void* stream);
+
+/*
+ * theta_residual -- residual of the scaled shared block ("The theta bundle" --
+ * Low-rank residual): R = W - diag(s) . W0, each element computed as one
+ * fused multiply-add fmaf(-s[o], W0[o,i], W[o,i]) and rounded once to dt.
+ *
+ *   weight, W0  device [O, I] of dt;  s device fp32 [O];  R device [O, I] of dt, written.
+ */
+int theta_residual(const void* weight, const void* W0, const float* s, int64_t O, int64_t I,
+                   theta_dtype dt, void* R, void* stream);
+
+/*
+ * theta_decompose_prelude -- the analytic decomposition of one projection
+ * family up to the truncated SVD ("The theta bundle" -- Analytic
+ * decomposition; "Banded sharing" for the bands): for each of the G bands of
+ * num_layers layers, W0[b] = band mean; then for every layer l of band b,
+ * s[l] = row scale of W_l against the stored W0[b] and, if residual is
+ * non-NULL, residual[l] = W_l - diag(s[l]) . W0[b]. Same arithmetic as the
+ * three calls above; the row scale and residual of a band's layers run in
+ * one pass that reads each W0[b] row once.
+ *
+ *   weights   host array of num_layers device pointers, each [O, I] of dt.
+ *   W0        host array of G device pointers, each [O, I] of dt, written.
+ *   s         host array of num_layers device pointers, each fp32 [O], written.
+ *   residual  host array of num_layers device pointers ([O, I] of dt, written),
+ *             or NULL to skip the residual.
+ * 1 <= G <= num_layers <= THETA_MAX_LAYERS.
+ */
+int theta_decompose_prelude(const void* const* weights, int num_layers, int G, int64_t O,
+                            int64_t I, theta_dtype dt, void* const* W0, float* const* s,
+                            void* const* residual, void* stream);
+
+/*
+ * theta_reconstruct -- reconstruct_weight(s, W0, U, V) = diag(s) . W0 + U . V^T
+ * ("The theta bundle" -- approximation formula; reconstruct_weight). fp32
+ * accumulation over the rank, one rounding to dt. rank == 0 leaves only the
+ * scaled shared block diag(s).W0 and allows U = V = NULL.
+ *
+ *   s fp32 [O]; W0 [O, I]; U [O, rank]; V [I, rank]; W_out [O, I], written.
+ *   All device pointers, dt elements except s.
+ */
+int theta_reconstruct(const float* s, const void* W0, const void* U, const void* V, int64_t O,
+                      int64_t I, int rank, theta_dtype dt, void* W_out, void* stream);
+
+/*
+ * theta_frob_error -- relative_frobenius_error(original, reconstructed)
+ * = ||A - B||_F / ||A||_F ("Quality" -- Reconstruction error; "The theta
+ * bundle" -- relative_frobenius_error). 0 if both norms are 0, +inf if only
+ * ||A|| is. Squares are summed in fp32 over 8-element groups and in fp64
+ * beyond; the two-stage reduction has a fixed order (deterministic).
+ *
+ *   original, reconstructed  device [n] of dt (any shape, flattened).
+ *   out        device double[1], written.
+ *   workspace  device scratch of at least theta_workspace_size(THETA_OP_FROB_ERROR)
+ *              bytes, 16-byte aligned; its contents are overwritten.
+ */
+int theta_frob_error(const void* original, const void* reconstructed, int64_t n, theta_dtype dt,
+                     double* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * theta_linear_forward -- the projection by the rebuilt weight without
+ * forming it:  Y = X . (diag(s) . W0 + U . V^T)^T = s (.) (X . W0^T) + (X . V) . U^T
+ * (identity from "The theta bundle" approximation formula).
+ *
+ *   X [M, I]; W0 [O, I] (the band's shared block); s fp32 [O]; U [O, rank];
+ *   V [I, rank]; Y [M, O], written. Device pointers, dt elements except s.
+ *   workspace  device scratch of theta_workspace_size(THETA_OP_LINEAR_FORWARD)
+ *              bytes (holds T = X . V); may be NULL when that size is 0.
+ * THETA_BF16: tensor cores (tcgen05) with fp32 accumulation in tensor memory;
+ * T = X.V is kept as a bf16 high part plus a bf16 low part, so the rank-r term
+ * carries about 16 significand bits. THETA_F32: fp32 CUDA cores throughout.
+ * rank == 0 allows U = V = NULL.
+ */
+int theta_linear_forward(const void* X, int64_t M, int64_t I, const void* W0, int64_t O,
+                         const float* s, const void* U, const void* V, int rank, theta_dtype dt,
+                         void* Y, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * theta_workspace_size -- device scratch bytes a call needs (0 if none).
+ * op is a theta_op; the sizes are those the call will receive (unused ones
+ * are ignored). Writes *bytes.
+ */
+int theta_workspace_size(int op, int64_t M, int64_t O, int64_t I, int rank, theta_dtype dt,
+                         size_t* bytes);
+
+/*
+ * theta_device_status -- synchronises `stream`, then reads and clears the
+ * current device's error flags. Returns THETA_ERR_TIMEOUT if a kernel's
+ * bounded wait ran out since the last check, THETA_ERR_CUDA on a CUDA error,
+ * else THETA_OK.
+ */
+int theta_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* THETA_H */

@@ -1,0 +1,110 @@
+// Shared device helpers for libtheta kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "theta.h"
+
+namespace theta {
+
+using bf16 = __nv_bfloat16;
+
+// Device error flags (one word per cause), set by bounded waits that ran out.
+enum : unsigned { ERR_WORD_TIMEOUT = 0, ERR_WORD_COUNT = 4 };
+
+// Upper bound of any single device wait, in nanoseconds of %globaltimer.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+
+// Pointer table passed by value as a kernel parameter.
+struct PtrTable {
+  const void* p[THETA_MAX_LAYERS];
+};
+struct MutPtrTable {
+  void* p[THETA_MAX_LAYERS];
+};
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void record_timeout(unsigned* err) {
+  if (err) atomicExch(err + ERR_WORD_TIMEOUT, 1u);
+}
+
+// ------------------------------------------------------------- element I/O
+// 16-byte vectors: 8 bf16 or 4 fp32 elements.
+template <typename T>
+struct Vec;
+template <>
+struct Vec<float> {
+  static constexpr int N = 4;
+  using raw = float4;
+};
+template <>
+struct Vec<bf16> {
+  static constexpr int N = 8;
+  using raw = uint4;
+};
+
+__device__ __forceinline__ void unpack(const float4& r, float (&f)[4]) {
+  f[0] = r.x; f[1] = r.y; f[2] = r.z; f[3] = r.w;
+}
+__device__ __forceinline__ void unpack(const uint4& r, float (&f)[8]) {
+  const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ float4 pack(const float (&f)[4], float4*) {
+  return make_float4(f[0], f[1], f[2], f[3]);
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint4 pack(const float (&f)[8], uint4*) {
+  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                    pack_bf16x2(f[6], f[7]));
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<bf16>(bf16 v) { return __bfloat162float(v); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float v);
+template <>
+__device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ bf16 from_f32<bf16>(float v) { return __float2bfloat16_rn(v); }
+
+// Read-only streaming load of 16 bytes (weights are read once per pass).
+template <typename R>
+__device__ __forceinline__ R ld_stream(const R* p) {
+  return __ldg(p);
+}
+
+// ------------------------------------------------------------- reductions
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace theta

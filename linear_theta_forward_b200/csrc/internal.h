@@ -1,0 +1,52 @@
+// Internal launcher declarations shared by the libtheta translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "theta.h"
+
+namespace theta {
+
+struct LaunchCtx {
+  cudaStream_t stream;
+  unsigned* err;  // device error words of the current device
+  int num_sms;
+  int device;
+};
+
+// ---- streaming kernels (stream_kernels.cu)
+cudaError_t launch_band_mean(const LaunchCtx& c, theta_dtype dt, const void* const* w, int n,
+                             int64_t O, int64_t I, void* W0);
+// Row scale of n layers against one W0 (a band), optionally with residuals.
+cudaError_t launch_rowscale_band(const LaunchCtx& c, theta_dtype dt, const void* W0,
+                                 const void* const* w, int n, int64_t O, int64_t I,
+                                 float* const* s, void* const* R);
+cudaError_t launch_residual(const LaunchCtx& c, theta_dtype dt, const void* w, const void* W0,
+                            const float* s, int64_t O, int64_t I, void* R);
+size_t frob_workspace_bytes();
+cudaError_t launch_frob(const LaunchCtx& c, theta_dtype dt, const void* a, const void* b,
+                        int64_t n, double* out, void* ws);
+
+// ---- CUDA-core GEMM paths (simt_kernels.cu): fp32 forward / reconstruct
+cudaError_t launch_xv_simt(const LaunchCtx& c, theta_dtype dt, const void* X, const void* V,
+                           int64_t M, int64_t I, int r, float* T);
+cudaError_t launch_forward_simt(const LaunchCtx& c, theta_dtype dt, const void* X,
+                                const void* W0, const float* s, const void* U, const float* T,
+                                int64_t M, int64_t O, int64_t I, int r, void* Y);
+cudaError_t launch_reconstruct_simt(const LaunchCtx& c, theta_dtype dt, const float* s,
+                                    const void* W0, const void* U, const void* V, int64_t O,
+                                    int64_t I, int r, void* W_out);
+
+// ---- tensor-core paths (umma_kernels.cu): bf16
+size_t forward_umma_workspace_bytes(int64_t M, int r);
+// Returns THETA_OK or a theta_status; CUDA errors are reported via *cuda_err.
+int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const float* s,
+                        const void* U, const void* V, int64_t M, int64_t O, int64_t I, int r,
+                        void* Y, void* ws, cudaError_t* cuda_err);
+int launch_reconstruct_umma(const LaunchCtx& c, const float* s, const void* W0, const void* U,
+                            const void* V, int64_t O, int64_t I, int r, void* W_out,
+                            cudaError_t* cuda_err);
+
+}  // namespace theta

@@ -1,0 +1,99 @@
+"""The C ABI on the host: loads, exports what include/theta.h declares, and
+validates arguments before touching a GPU (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle_checks as oc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "theta.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(theta_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ["theta_band_index", "theta_band_mean", "theta_row_scale", "theta_residual",
+                     "theta_decompose_prelude", "theta_reconstruct", "theta_frob_error",
+                     "theta_linear_forward", "theta_workspace_size", "theta_device_status"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(raw, name), f"{name} declared in theta.h but not exported"
+
+
+def test_binding_names_match_c_names(lib):
+    for name in declared_functions():
+        assert callable(getattr(lib, name)), name
+
+
+def test_version_and_status_strings(lib):
+    assert lib.theta_version() == 1
+    assert lib.theta_status_string(0) == "THETA_OK"
+    assert lib.theta_status_string(-5) == "THETA_ERR_TIMEOUT"
+    assert lib.theta_status_string(12345) == "THETA_ERR_UNKNOWN"
+
+
+@pytest.mark.parametrize("L,G", [(4, 2), (26, 1), (26, 4), (26, 7), (26, 26), (60, 15), (60, 4), (1, 1),
+                                 (256, 3), (97, 13)])
+def test_band_index_matches_oracle_bit_exactly(lib, L, G):
+    bol, start = lib.theta_band_index(L, G)
+    obol, ostart = oracle.band_index(L, G)
+    assert bol.dtype == np.int32 and np.array_equal(bol, obol)
+    assert np.array_equal(start, ostart)
+
+
+def test_band_index_golden_table(lib):
+    for L, G, sizes in oc.read_band_golden():
+        _, start = lib.theta_band_index(L, G)
+        assert list(np.diff(start)) == sizes
+
+
+@pytest.mark.parametrize("L,G", [(4, 0), (4, 5), (0, 1), (-1, 1), (3, -2)])
+def test_band_index_rejects(lib, L, G):
+    with pytest.raises(lib.ThetaError) as e:
+        lib.theta_band_index(L, G)
+    assert e.value.status == -1
+    assert "G" in lib.theta_last_error()
+
+
+def test_validation_happens_before_any_cuda_call(lib):
+    raw = lib.lib
+    # each call below has an argument error; none may reach the CUDA runtime
+    assert raw.theta_band_mean(None, 0, 4, 4, 0, None, None) == -1
+    assert raw.theta_band_mean(None, 1, 4, 4, 7, None, None) == -1           # bad dtype
+    assert raw.theta_row_scale(None, None, 0, 4, 0, None, None) == -1
+    assert raw.theta_residual(None, None, None, 4, 4, 0, None, None) == -1
+    assert raw.theta_decompose_prelude(None, 4, 5, 8, 8, 0, None, None, None, None) == -1
+    assert raw.theta_decompose_prelude(None, 300, 1, 8, 8, 0, None, None, None, None) == -1
+    assert raw.theta_reconstruct(None, None, None, None, 8, 8, -1, 0, None, None) == -1
+    assert raw.theta_frob_error(None, None, -1, 0, None, None, 0, None) == -1
+    assert raw.theta_frob_error(None, None, 0, 0, ctypes.c_void_p(16), None, 0, None) == -6
+    assert raw.theta_linear_forward(None, 0, 8, None, 8, None, None, None, 0, 0, None, None, 0, None) == -1
+    assert raw.theta_linear_forward(ctypes.c_void_p(16), 4, 8, ctypes.c_void_p(16), 8, ctypes.c_void_p(16),
+                                    None, None, 8, 0, ctypes.c_void_p(16), None, 0, None) == -1  # rank>0, U NULL
+    assert raw.theta_linear_forward(ctypes.c_void_p(16), 4, 8, ctypes.c_void_p(16), 8, ctypes.c_void_p(16),
+                                    ctypes.c_void_p(16), ctypes.c_void_p(16), 8, 1, ctypes.c_void_p(16),
+                                    None, 0, None) == -6                                         # no workspace
+
+
+def test_workspace_sizes(lib):
+    assert lib.theta_workspace_size(lib.THETA_OP_FROB_ERROR, 1, 1, 1, 0, lib.THETA_F32) >= 16
+    assert lib.theta_workspace_size(lib.THETA_OP_LINEAR_FORWARD, 16, 256, 256, 0, lib.THETA_F32) == 0
+    for dt in (lib.THETA_F32, lib.THETA_BF16):
+        b = lib.theta_workspace_size(lib.THETA_OP_LINEAR_FORWARD, 300, 64, 64, 24, dt)
+        assert b >= 300 * 24 * 4 and b % 256 == 0
+    with pytest.raises(lib.ThetaError):
+        lib.theta_workspace_size(99, 1, 1, 1, 0, lib.THETA_F32)
