@@ -551,6 +551,80 @@ def run_e2e(torch, theta, wl, run, stream, step_bytes, steps, world):
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ms, 3), "steps": steps}
 
 
+def run_op(args):
+    """One entry point on one synthetic problem, timed per call with CUDA
+    events (median of --iters calls, L2 flushed before each). Prints a JSON
+    line with the achieved rate and its fraction of the measured roofline."""
+    import torch
+    torch.cuda.set_device(0)
+    import linear_theta_forward_b200 as theta
+    peaks = measured_peaks()
+    M, O, I, r, L, G = args.M, args.O, args.I, args.rank, args.layers, args.G
+    seed = 0
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    if args.op == "forward":
+        X = syn.device_normal((M, I), 1.0, seed, "X", M, I)
+        W0 = syn.device_normal((O, I), 0.02, seed, "W0", O, I)
+        s = 1.0 + syn.device_normal((O,), 0.05, seed, "s", O, dtype="f32")
+        U = syn.device_normal((O, r), 0.01, seed, "U", O, r) if r else None
+        V = syn.device_normal((I, r), 0.01, seed, "V", I, r) if r else None
+        Y = torch.empty(M, O, dtype=torch.bfloat16, device="cuda")
+        nb = theta.theta_workspace_size(theta.THETA_OP_LINEAR_FORWARD, M, O, I, r, theta.THETA_BF16)
+        ws = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
+        call = lambda: theta.theta_linear_forward(X, W0, s, U, V, Y, ws)  # noqa: E731
+        nbytes, nflops = bytes_forward(M, O, I, r), flops_forward(M, O, I, r)
+    elif args.op == "reconstruct":
+        W0 = syn.device_normal((O, I), 0.02, seed, "W0", O, I)
+        s = 1.0 + syn.device_normal((O,), 0.05, seed, "s", O, dtype="f32")
+        U = syn.device_normal((O, r), 0.01, seed, "U", O, r) if r else None
+        V = syn.device_normal((I, r), 0.01, seed, "V", I, r) if r else None
+        out = torch.empty(O, I, dtype=torch.bfloat16, device="cuda")
+        call = lambda: theta.theta_reconstruct(s, W0, U, V, out)  # noqa: E731
+        nbytes, nflops = bytes_reconstruct(O, I, r), 2 * O * I * r
+    elif args.op == "prelude":
+        W = syn.device_family_weights(L, O, I, seed=seed, family="op")
+        W0 = [torch.empty(O, I, dtype=torch.bfloat16, device="cuda") for _ in range(G)]
+        sl = [torch.empty(O, dtype=torch.float32, device="cuda") for _ in range(L)]
+        R = [torch.empty(O, I, dtype=torch.bfloat16, device="cuda") for _ in range(L)]
+        call = lambda: theta.theta_decompose_prelude(W, G, W0, sl, R)  # noqa: E731
+        nbytes, nflops = bytes_band_mean(L, G, O, I) + bytes_rowscale_residual(L, G, O, I), 0
+    elif args.op == "frob":
+        A = syn.device_normal((O, I), 0.02, seed, "A", O, I)
+        B = syn.device_normal((O, I), 0.02, seed, "B", O, I)
+        out = torch.empty(1, dtype=torch.float64, device="cuda")
+        ws = torch.empty(theta.theta_workspace_size(theta.THETA_OP_FROB_ERROR, 1, 1, 1, 0, 1), dtype=torch.uint8,
+                         device="cuda")
+        call = lambda: theta.theta_frob_error(A, B, out, ws)  # noqa: E731
+        nbytes, nflops = bytes_frob(O, I), 0
+    else:
+        raise ValueError(args.op)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    theta.theta_device_status()
+    times = []
+    for _ in range(args.iters):
+        flush.fill_(1)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        call()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    theta.theta_device_status()
+    ms = statistics.median(times)
+    line = {"op": args.op, "shape": {"M": M, "O": O, "I": I, "rank": r, "layers": L, "G": G}, "dtype": "bf16",
+            "ms": round(ms, 5), "iters": args.iters, "l2": "flushed (256 MiB write) before every call",
+            "GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1),
+            "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4), "algorithmic_bytes": nbytes}
+    if nflops:
+        line["TFLOP/s"] = round(nflops / (ms * 1e-3) / 1e12, 2)
+        line["frac_tensor_burst"] = round(nflops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -563,7 +637,18 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-rows", type=int, default=32)
+    ap.add_argument("--op", choices=["forward", "reconstruct", "prelude", "frob"],
+                    help="time one entry point on one problem instead of the whole step")
+    ap.add_argument("--M", type=int, default=256)
+    ap.add_argument("--O", type=int, default=21504)
+    ap.add_argument("--I", type=int, default=5376)
+    ap.add_argument("--rank", type=int, default=64)
+    ap.add_argument("--layers", type=int, default=4)
+    ap.add_argument("--G", type=int, default=1)
+    ap.add_argument("--iters", type=int, default=20)
     args = ap.parse_args(argv)
+    if args.op:
+        return run_op(args)
     if args.warmup < 3 and args.impl == "native":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
