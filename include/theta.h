@@ -189,6 +189,36 @@ int theta_linear_forward(const void* X, int64_t M, int64_t I, const void* W0, in
                          void* Y, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * theta_linear_forward_noalloc -- theta_linear_forward for callers that
+ * cannot allocate device memory. (A library convenience: the pages describe
+ * no counterpart.)
+ *
+ * Same arguments, arithmetic, kernels and result as theta_linear_forward,
+ * minus the workspace: its scratch (T = X.V) lives in a 4 MiB array built
+ * into the library. It is meant for code that must not call cudaMalloc:
+ * work recorded into a CUDA graph (allocation is not allowed during stream
+ * capture), engines whose device memory is all owned by their own fixed
+ * pool, and plugins that are handed only input and output buffers.
+ *
+ *   - Capacity: the call needs theta_workspace_size(THETA_OP_LINEAR_FORWARD)
+ *     bytes, at most 4 MiB (about M * rank <= 1,048,576). Larger requests
+ *     return THETA_ERR_WORKSPACE before anything is enqueued.
+ *   - Memory: every GPU that loads the library holds the 4 MiB array until
+ *     the process exits. This entry point itself allocates nothing.
+ *   - Sharing: all calls on a device use the same array. Calls ordered on one
+ *     stream are safe; calls whose kernels may overlap on the GPU (different
+ *     streams without ordering between them) race on it and must not be made.
+ *     Each call writes the scratch it reads, so leftovers from an earlier call
+ *     do not matter.
+ *   - Set-up: the first call on each device looks up the array's device
+ *     address (cudaGetSymbolAddress, with that device current). Make that
+ *     first call before any stream capture begins.
+ */
+int theta_linear_forward_noalloc(const void* X, int64_t M, int64_t I, const void* W0, int64_t O,
+                                 const float* s, const void* U, const void* V, int rank,
+                                 theta_dtype dt, void* Y, void* stream);
+
+/*
  * theta_workspace_size -- device scratch bytes a call needs (0 if none).
  * op is a theta_op; the sizes are those the call will receive (unused ones
  * are ignored). Writes *bytes.

@@ -19,7 +19,7 @@ __all__ = [
     "theta_version", "theta_status_string", "theta_last_error", "theta_band_index",
     "theta_band_mean", "theta_row_scale", "theta_residual", "theta_decompose_prelude",
     "theta_reconstruct", "theta_frob_error", "theta_linear_forward", "theta_workspace_size",
-    "theta_device_status",
+    "theta_device_status", "theta_linear_forward_noalloc",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtheta.so")
@@ -58,6 +58,7 @@ _sig("theta_reconstruct", _int, _vp, _vp, _vp, _vp, _i64, _i64, _int, _int, _vp,
 _sig("theta_frob_error", _int, _vp, _vp, _i64, _int, _vp, _vp, _sz, _vp)
 _sig("theta_linear_forward", _int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp,
      _sz, _vp)
+_sig("theta_linear_forward_noalloc", _int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp)
 _sig("theta_workspace_size", _int, _int, _i64, _i64, _i64, _int, _int, ctypes.POINTER(_sz))
 _sig("theta_device_status", _int, _vp)
 
@@ -214,6 +215,19 @@ def theta_linear_forward(X, W0, s, U, V, Y, workspace=None, stream=None) -> None
                                     _ptr(U, "U", optional=True), _ptr(V, "V", optional=True), rank,
                                     _dtype_code(X), _ptr(Y, "Y"), ws_ptr, ws_bytes, _stream(stream)),
            "theta_linear_forward")
+
+
+def theta_linear_forward_noalloc(X, W0, s, U, V, Y, stream=None) -> None:
+    """theta_linear_forward without a workspace argument: the scratch is the
+    library's built-in array (for callers that cannot allocate device memory;
+    see include/theta.h for its capacity and sharing rules)."""
+    M, I = X.shape
+    O = W0.shape[0]
+    rank = 0 if U is None else U.shape[1]
+    _check(lib.theta_linear_forward_noalloc(_ptr(X, "X"), M, I, _ptr(W0, "W0"), O, _ptr(s, "s"),
+                                            _ptr(U, "U", optional=True), _ptr(V, "V", optional=True), rank,
+                                            _dtype_code(X), _ptr(Y, "Y"), _stream(stream)),
+           "theta_linear_forward_noalloc")
 
 
 def theta_device_status(stream=None) -> None:

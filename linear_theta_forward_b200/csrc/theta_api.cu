@@ -88,6 +88,13 @@ size_t forward_ws_bytes(int64_t M, int r, theta_dtype dt) {
   } while (0)
 
 }  // namespace
+
+// Lets other translation units report through theta_last_error().
+int report_error(int status, const char* message) {
+  t_last_error = message;
+  return status;
+}
+
 }  // namespace theta
 
 using namespace theta;
