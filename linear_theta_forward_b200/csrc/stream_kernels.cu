@@ -34,6 +34,7 @@ int grid_for(const LaunchCtx& c, int64_t work_items, int per_block, int blocks_p
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 band_mean_kernel(PtrTable src, int n, int64_t nvec, int64_t count, T* __restrict__ out) {
+  pdl_enter();
   using V = Vec<T>;
   using R = typename V::raw;
   const float fn = (float)n;
@@ -84,6 +85,7 @@ template <typename T, int TPR, int VPT>
 __global__ void __launch_bounds__(kThreads)
 rowscale_band_kernel(const T* __restrict__ W0, PtrTable w, MutPtrTable s_out, MutPtrTable r_out,
                      int n, int64_t O, int64_t I, int write_r) {
+  pdl_enter();
   using V = Vec<T>;
   using R = typename V::raw;
   constexpr int GROUPS = kThreads / TPR;
@@ -169,6 +171,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 rowscale_band_scalar_kernel(const T* __restrict__ W0, PtrTable w, MutPtrTable s_out,
                             MutPtrTable r_out, int n, int64_t O, int64_t I, int write_r) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
   for (int64_t o = (int64_t)blockIdx.x * (kThreads / 32) + threadIdx.x / 32; o < O; o += warps) {
@@ -198,6 +201,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 residual_vec_kernel(const T* __restrict__ w, const T* __restrict__ W0, const float* __restrict__ s,
                     int64_t nv_row, int64_t nvec, T* __restrict__ R) {
+  pdl_enter();
   using V = Vec<T>;
   using Rw = typename V::raw;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -216,6 +220,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 residual_scalar_kernel(const T* __restrict__ w, const T* __restrict__ W0, const float* __restrict__ s,
                        int64_t I, int64_t count, T* __restrict__ R) {
+  pdl_enter();
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += stride)
     R[i] = from_f32<T>(fmaf(-s[i / I], to_f32(W0[i]), to_f32(w[i])));
@@ -228,6 +233,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 frob_partial_kernel(const T* __restrict__ A, const T* __restrict__ B, int64_t nvec, int64_t count,
                     double* __restrict__ ws) {
+  pdl_enter();
   using V = Vec<T>;
   using R = typename V::raw;
   double num = 0.0, den = 0.0;
@@ -273,6 +279,7 @@ frob_partial_kernel(const T* __restrict__ A, const T* __restrict__ B, int64_t nv
 
 __global__ void __launch_bounds__(kThreads) frob_final_kernel(const double* __restrict__ ws, int nb,
                                                               double* __restrict__ out) {
+  pdl_enter();
   double num = 0.0, den = 0.0;
   for (int k = threadIdx.x; k < nb; k += blockDim.x) {
     num += ws[2 * k];
@@ -313,28 +320,30 @@ cudaError_t band_mean_t(const LaunchCtx& c, const void* const* w, int n, int64_t
   const int64_t count = O * I;
   const int64_t nvec = ok ? count / Vec<T>::N : 0;
   const int grid = grid_for(c, ok ? nvec : count, kThreads, 8);
-  band_mean_kernel<T><<<grid, kThreads, 0, c.stream>>>(tab, n, nvec, count, static_cast<T*>(W0));
-  return cudaGetLastError();
+  return launch_pdl(band_mean_kernel<T>, grid, kThreads, 0, c.stream, 1, tab, n, nvec, count, static_cast<T*>(W0));
 }
 
 template <typename T, int TPR, int VPT>
-void launch_rs(const LaunchCtx& c, int grid, const T* W0, const PtrTable& w, const MutPtrTable& s,
-               const MutPtrTable& r, int n, int64_t O, int64_t I, int write_r) {
-  rowscale_band_kernel<T, TPR, VPT><<<grid, kThreads, 0, c.stream>>>(W0, w, s, r, n, O, I, write_r);
+cudaError_t launch_rs(const LaunchCtx& c, int grid, const T* W0, const PtrTable& w, const MutPtrTable& s,
+                      const MutPtrTable& r, int n, int64_t O, int64_t I, int write_r) {
+  return launch_pdl(rowscale_band_kernel<T, TPR, VPT>, grid, kThreads, 0, c.stream, 1, W0, w, s, r, n, O, I,
+                    write_r);
 }
 
+// Launches the register-resident row-scale variant for (TPR, vpt); returns
+// false if no such variant exists.
 template <typename T, int TPR>
 bool dispatch_vpt(const LaunchCtx& c, int vpt, int grid, const T* W0, const PtrTable& w,
                   const MutPtrTable& s, const MutPtrTable& r, int n, int64_t O, int64_t I,
-                  int write_r) {
+                  int write_r, cudaError_t* e) {
   switch (vpt) {
-    case 1: launch_rs<T, TPR, 1>(c, grid, W0, w, s, r, n, O, I, write_r); return true;
-    case 2: launch_rs<T, TPR, 2>(c, grid, W0, w, s, r, n, O, I, write_r); return true;
-    case 3: launch_rs<T, TPR, 3>(c, grid, W0, w, s, r, n, O, I, write_r); return true;
-    case 4: launch_rs<T, TPR, 4>(c, grid, W0, w, s, r, n, O, I, write_r); return true;
-    case 6: launch_rs<T, TPR, 6>(c, grid, W0, w, s, r, n, O, I, write_r); return true;
-    case 8: launch_rs<T, TPR, 8>(c, grid, W0, w, s, r, n, O, I, write_r); return true;
-    case 12: launch_rs<T, TPR, 12>(c, grid, W0, w, s, r, n, O, I, write_r); return true;
+    case 1: *e = launch_rs<T, TPR, 1>(c, grid, W0, w, s, r, n, O, I, write_r); return true;
+    case 2: *e = launch_rs<T, TPR, 2>(c, grid, W0, w, s, r, n, O, I, write_r); return true;
+    case 3: *e = launch_rs<T, TPR, 3>(c, grid, W0, w, s, r, n, O, I, write_r); return true;
+    case 4: *e = launch_rs<T, TPR, 4>(c, grid, W0, w, s, r, n, O, I, write_r); return true;
+    case 6: *e = launch_rs<T, TPR, 6>(c, grid, W0, w, s, r, n, O, I, write_r); return true;
+    case 8: *e = launch_rs<T, TPR, 8>(c, grid, W0, w, s, r, n, O, I, write_r); return true;
+    case 12: *e = launch_rs<T, TPR, 12>(c, grid, W0, w, s, r, n, O, I, write_r); return true;
   }
   return false;
 }
@@ -377,18 +386,18 @@ cudaError_t rowscale_t(const LaunchCtx& c, const void* W0, const void* const* w,
     const int grid = grid_for(c, O, groups, vpt <= 4 ? 8 : 4);
     const T* W0t = static_cast<const T*>(W0);
     bool launched = false;
+    cudaError_t e = cudaSuccess;
     switch (tpr) {
-      case 32: launched = dispatch_vpt<T, 32>(c, vpt, grid, W0t, wt, st, rt, n, O, I, write_r); break;
-      case 64: launched = dispatch_vpt<T, 64>(c, vpt, grid, W0t, wt, st, rt, n, O, I, write_r); break;
-      case 128: launched = dispatch_vpt<T, 128>(c, vpt, grid, W0t, wt, st, rt, n, O, I, write_r); break;
-      case 256: launched = dispatch_vpt<T, 256>(c, vpt, grid, W0t, wt, st, rt, n, O, I, write_r); break;
+      case 32: launched = dispatch_vpt<T, 32>(c, vpt, grid, W0t, wt, st, rt, n, O, I, write_r, &e); break;
+      case 64: launched = dispatch_vpt<T, 64>(c, vpt, grid, W0t, wt, st, rt, n, O, I, write_r, &e); break;
+      case 128: launched = dispatch_vpt<T, 128>(c, vpt, grid, W0t, wt, st, rt, n, O, I, write_r, &e); break;
+      case 256: launched = dispatch_vpt<T, 256>(c, vpt, grid, W0t, wt, st, rt, n, O, I, write_r, &e); break;
     }
-    if (launched) return cudaGetLastError();
+    if (launched) return e;
   }
   const int grid = grid_for(c, O, kThreads / 32, 8);
-  rowscale_band_scalar_kernel<T><<<grid, kThreads, 0, c.stream>>>(static_cast<const T*>(W0), wt, st,
-                                                                  rt, n, O, I, write_r);
-  return cudaGetLastError();
+  return launch_pdl(rowscale_band_scalar_kernel<T>, grid, kThreads, 0, c.stream, 1, static_cast<const T*>(W0),
+                    wt, st, rt, n, O, I, write_r);
 }
 
 template <typename T>
@@ -398,13 +407,12 @@ cudaError_t residual_t(const LaunchCtx& c, const void* w, const void* W0, const 
   const int64_t count = O * I;
   if (vec) {
     const int64_t nvec = count / Vec<T>::N;
-    residual_vec_kernel<T><<<grid_for(c, nvec, kThreads, 8), kThreads, 0, c.stream>>>(
-        static_cast<const T*>(w), static_cast<const T*>(W0), s, I / Vec<T>::N, nvec, static_cast<T*>(R));
-  } else {
-    residual_scalar_kernel<T><<<grid_for(c, count, kThreads, 8), kThreads, 0, c.stream>>>(
-        static_cast<const T*>(w), static_cast<const T*>(W0), s, I, count, static_cast<T*>(R));
+    return launch_pdl(residual_vec_kernel<T>, grid_for(c, nvec, kThreads, 8), kThreads, 0, c.stream, 1,
+                      static_cast<const T*>(w), static_cast<const T*>(W0), s, I / Vec<T>::N, nvec,
+                      static_cast<T*>(R));
   }
-  return cudaGetLastError();
+  return launch_pdl(residual_scalar_kernel<T>, grid_for(c, count, kThreads, 8), kThreads, 0, c.stream, 1,
+                    static_cast<const T*>(w), static_cast<const T*>(W0), s, I, count, static_cast<T*>(R));
 }
 
 template <typename T>
@@ -415,10 +423,10 @@ cudaError_t frob_t(const LaunchCtx& c, const void* a, const void* b, int64_t n, 
   int grid = grid_for(c, vec ? nvec : n, kThreads, 4);
   if (grid > kFrobMaxBlocks) grid = kFrobMaxBlocks;
   double* part = static_cast<double*>(ws);
-  frob_partial_kernel<T><<<grid, kThreads, 0, c.stream>>>(static_cast<const T*>(a),
-                                                          static_cast<const T*>(b), nvec, n, part);
-  frob_final_kernel<<<1, kThreads, 0, c.stream>>>(part, grid, out);
-  return cudaGetLastError();
+  cudaError_t e = launch_pdl(frob_partial_kernel<T>, grid, kThreads, 0, c.stream, 1, static_cast<const T*>(a),
+                             static_cast<const T*>(b), nvec, n, part);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(frob_final_kernel, 1, kThreads, 0, c.stream, 1, static_cast<const double*>(part), grid, out);
 }
 
 }  // namespace

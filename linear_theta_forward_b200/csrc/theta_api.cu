@@ -70,7 +70,6 @@ int make_ctx(void* stream, LaunchCtx* ctx) {
 }
 
 bool valid_dt(theta_dtype dt) { return dt == THETA_F32 || dt == THETA_BF16; }
-size_t elem_size(theta_dtype dt) { return dt == THETA_BF16 ? 2 : 4; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 

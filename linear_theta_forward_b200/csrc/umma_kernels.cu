@@ -8,15 +8,23 @@
 //   warp 0  TMA producer (one lane)
 //   warp 1  tensor-memory allocator and MMA issuer (one lane)
 //   warps 2-5  epilogue: tcgen05.ld of their 32-lane quarter of D1/D2
-// Three epilogues ("The theta bundle" -- approximation formula):
+// Two epilogues ("The theta bundle" -- approximation formula):
 //   FORWARD  Y[m, o] = s[o] * D1[o, m] + D2[o, m]   with A1 = W0, B1 = X,
 //            A2 = U, B2/B3 = high/low bf16 parts of T = X.V  (swap-AB: the
 //            weight rows fill the 128-row MMA side, tokens are N)
 //   XV       T_hi/T_lo[m, j] from D1[m, j]           with A1 = X, B1 = V (MN-major)
-//   RECON    W[o, i] = s[o] * W0[o, i] + D1[o, i]   with A1 = U, B1 = V (K = rank)
-// Decode-sized problems split K across the CTAs of a thread-block cluster;
-// the partial tiles are summed in a fixed order through distributed shared
-// memory (deterministic, no global scratch).
+// When the tiles alone cannot fill the GPU, K is split across the CTAs of a
+// thread-block cluster (up to 16); the partial tiles are summed in a fixed
+// order through distributed shared memory (deterministic, no global scratch).
+//
+// reconstruct_weight has its own kernel (recon_kernel): the K = rank MMA
+// U.V^T into tensor memory, the W0 tile brought in by TMA next to U and V,
+// s*W0 + U.V^T combined in swizzled shared memory and written back by a TMA
+// store, so both HBM streams (W0 in, W out) move as whole tiles.
+//
+// All kernels are launched with programmatic dependent launch: their
+// prologue (barrier init, tensor-memory allocation) overlaps the previous
+// kernel, and griddepcontrol.wait precedes every global memory access.
 //
 // Every wait is bounded (kWaitLimitNs); a wait that gives up records a
 // device error flag, raises a CTA-wide abort so the other roles stop, and the
@@ -33,7 +41,7 @@ namespace theta {
 
 namespace {
 
-enum Mode { MODE_FORWARD = 0, MODE_XV = 1, MODE_RECON = 2 };
+enum Mode { MODE_FORWARD = 0, MODE_XV = 1 };
 
 constexpr int kThreads = 192;
 constexpr int kBM = 128;       // MMA M (rows of A)
@@ -43,13 +51,12 @@ constexpr int kPitch = 129;    // fp32 pitch of the split-K partial tiles (bank-
 
 struct Args {
   int rows;        // valid rows of the A side (O, or M tokens for XV)
-  int cols;        // valid columns of the B side (M tokens, I, or rank)
+  int cols;        // valid columns of the B side (M tokens, or rank)
   int kb1;         // K blocks of phase 1
   int kb2;         // K blocks of phase 2 (0: none)
   int splits;      // cluster size along x (split-K)
-  const float* s;  // FORWARD / RECON row scale
-  const bf16* W0;  // RECON
-  bf16* out;       // FORWARD: Y [cols, rows]; RECON: W [rows, cols]
+  const float* s;  // FORWARD row scale
+  bf16* out;       // FORWARD: Y [cols, rows]
   bf16* t_hi;      // XV outputs [rows, r]
   bf16* t_lo;
   int r;
@@ -60,7 +67,8 @@ template <int BN, int MODE>
 struct Cfg {
   static constexpr int kBBytes = BN * kBK * 2;  // XV: BN = padded rank, MN-major atoms of 64 columns
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = BN <= 32 ? 8 : (BN <= 64 ? 6 : 4);
+  // small rings for small BN so 2-3 decode CTAs share an SM
+  static constexpr int kStages = (BN == 128 || (MODE == MODE_XV && BN > 128)) ? 3 : 4;
   static constexpr int kTmemNeed = MODE == MODE_FORWARD ? 2 * BN : BN;
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
@@ -70,7 +78,7 @@ struct Cfg {
 };
 
 template <int BN, int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads)
 umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
             const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
             const __grid_constant__ CUtensorMap tmB3, const Args args) {
@@ -113,6 +121,7 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_enter();
 
   auto give_up = [&]() {
     record_timeout(args.err);
@@ -210,14 +219,15 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // accumulator row = TMEM lane
     const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
-    const bool ok = ptx::mbar_wait(accum, 0, abort_flag);
+    bool ok = ptx::mbar_wait(accum, 0, abort_flag);
     if (!ok) give_up();
+    ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
     ptx::tc_fence_after();
     const int grow = m_tile * kBM + row;  // global row of A
     const int col0 = n_tile * BN;
     const int ncols = min(BN, args.cols - col0);
     float so = 0.f;
-    if constexpr (MODE != MODE_XV) so = (grow < args.rows) ? __ldg(args.s + grow) : 0.f;
+    if constexpr (MODE == MODE_FORWARD) so = (grow < args.rows) ? __ldg(args.s + grow) : 0.f;
     float* part = reinterpret_cast<float*>(smem);
     if (ok) {
       for (int c0 = 0; c0 < ncols; c0 += 16) {
@@ -251,23 +261,6 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
                 args.t_hi[(int64_t)grow * args.r + j] = hi;
                 args.t_lo[(int64_t)grow * args.r + j] = __float2bfloat16_rn(d1[e] - __bfloat162float(hi));
               }
-            }
-          } else {  // RECON: 16 consecutive columns of one weight row
-            const int64_t base = (int64_t)grow * args.cols + col0 + c0;
-            if (c0 + 16 <= ncols) {
-              const uint4* w0v = reinterpret_cast<const uint4*>(args.W0 + base);
-              uint4* ov = reinterpret_cast<uint4*>(args.out + base);
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                float w[8], o[8];
-                unpack(__ldg(w0v + h), w);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) o[e] = fmaf(so, w[e], d1[8 * h + e]);
-                ov[h] = pack(o, (uint4*)nullptr);
-              }
-            } else {
-              for (int e = 0; e < ncols - c0; ++e)
-                args.out[base + e] = __float2bfloat16_rn(fmaf(so, __bfloat162float(args.W0[base + e]), d1[e]));
             }
           }
         }
@@ -315,6 +308,7 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
 // s (.) W0 for rank 0 (no tensor-core work).
 __global__ void __launch_bounds__(256) scale_rows_kernel(const float* __restrict__ s, const bf16* __restrict__ W0,
                                                          int64_t I, int64_t nvec, bf16* __restrict__ out) {
+  pdl_enter();
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t per_row = I / 8;
   for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < nvec; v += stride) {
@@ -325,6 +319,142 @@ __global__ void __launch_bounds__(256) scale_rows_kernel(const float* __restrict
     for (int e = 0; e < 8; ++e) o[e] = sc * w[e];
     reinterpret_cast<uint4*>(out)[v] = pack(o, (uint4*)nullptr);
   }
+}
+
+// ------------------------------------------------------------- reconstruct
+// One 128 x 128 tile of W = diag(s).W0 + U.V^T. 128 threads: thread 0 issues
+// the TMA loads (U and V rank blocks on one barrier, the W0 tile on another)
+// and the final TMA store; thread 32 issues the K = rank MMAs; then all four
+// warps read their 32-lane quarter of U.V^T from tensor memory, combine it
+// with s * W0 in place in the swizzled W0 tile, and the tile is stored.
+constexpr int kRecThreads = 128;
+constexpr int kRecN = 128;  // columns of W per tile
+
+template <int KB>
+struct RecCfg {
+  static constexpr int kOpBytes = KB * kABytes;         // U or V: KB blocks of 128 rows x 64
+  static constexpr int kWBytes = 2 * kABytes;           // W0 / output tile: two 64-column boxes
+  static constexpr int kSmemBytes = 2 * kOpBytes + kWBytes + 1024 + 128;
+};
+
+template <int KB>
+__global__ void __launch_bounds__(kRecThreads)
+recon_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CUtensorMap tmV,
+             const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ CUtensorMap tmOut,
+             const float* __restrict__ s, int O, int I, unsigned* err) {
+  using C = RecCfg<KB>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sU = smem;
+  uint8_t* sV = smem + C::kOpBytes;
+  uint8_t* sW = sV + C::kOpBytes;
+  uint64_t* bar_uv = reinterpret_cast<uint64_t*>(sW + C::kWBytes);
+  uint64_t* bar_w = bar_uv + 1;
+  uint64_t* bar_acc = bar_w + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_acc + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int i0 = blockIdx.x * kRecN, o0 = blockIdx.y * kBM;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar_uv, 1);
+    ptx::mbar_init(bar_w, 1);
+    ptx::mbar_init(bar_acc, 1);
+    *abort_flag = 0;
+    ptx::fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, kRecN);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_enter();
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_arrive_expect_tx(bar_uv, 2 * C::kOpBytes);
+#pragma unroll
+    for (int kb = 0; kb < KB; ++kb) {
+      ptx::tma_load_2d(sU + kb * kABytes, &tmU, bar_uv, kb * kBK, o0);
+      ptx::tma_load_2d(sV + kb * kABytes, &tmV, bar_uv, kb * kBK, i0);
+    }
+    ptx::mbar_arrive_expect_tx(bar_w, C::kWBytes);
+    ptx::tma_load_2d(sW, &tmW0, bar_w, i0, o0);
+    ptx::tma_load_2d(sW + kABytes, &tmW0, bar_w, i0 + kBK, o0);
+  }
+  bool mma_issued = false;
+  if (threadIdx.x == 32) {
+    if (ptx::mbar_wait(bar_uv, 0, abort_flag)) {
+      ptx::tc_fence_after();
+      constexpr uint32_t idesc = ptx::idesc_bf16(kBM, kRecN, 0);
+      const uint32_t ua = ptx::smem_u32(sU), va = ptx::smem_u32(sV);
+#pragma unroll
+      for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk)
+          ptx::umma_bf16(tmem, ptx::sdesc_sw128(ua + kb * kABytes + kk * 32, 16, 1024),
+                         ptx::sdesc_sw128(va + kb * kABytes + kk * 32, 16, 1024), idesc, (kb | kk) ? 1u : 0u);
+      ptx::umma_commit(bar_acc);
+      mma_issued = true;
+    } else {
+      record_timeout(err);
+      *abort_flag = 1;
+    }
+  }
+
+  // epilogue: warp w owns tensor-memory lanes (rows) 32w .. 32w+31
+  const int row = warp * 32 + lane;
+  bool ok = ptx::mbar_wait(bar_acc, 0, abort_flag) && ptx::mbar_wait(bar_w, 0, abort_flag);
+  if (!ok && !*abort_flag) {
+    record_timeout(err);
+    *abort_flag = 1;
+  }
+  ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+  ptx::tc_fence_after();
+  const float so = (o0 + row < O) ? __ldg(s + o0 + row) : 0.f;
+  const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
+  if (ok) {
+#pragma unroll 1
+    for (int c0 = 0; c0 < kRecN; c0 += 16) {
+      float d[16];
+      ptx::tmem_ld16(taddr + c0, d);
+      ptx::tmem_wait_ld();
+      uint8_t* rowp = sW + (c0 / kBK) * kABytes + row * 128;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int chunk = ((c0 % kBK) / 8 + h) ^ (row & 7);  // 128-byte swizzle of 16-byte chunks
+        uint4* p = reinterpret_cast<uint4*>(rowp + chunk * 16);
+        float w[8], o[8];
+        unpack(*p, w);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = fmaf(so, w[e], d[8 * h + e]);
+        *p = pack(o, (uint4*)nullptr);
+      }
+    }
+  }
+  ptx::fence_proxy_async_smem();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    if (!*abort_flag) {
+      ptx::tma_store_2d(&tmOut, sW, i0, o0);
+      if (i0 + kBK < I) ptx::tma_store_2d(&tmOut, sW + kABytes, i0 + kBK, o0);
+      ptx::bulk_commit();
+      ptx::bulk_wait_read();
+    } else {
+      int never = 0;  // drain the loads before shared memory goes away
+      ptx::mbar_wait(bar_uv, 0, &never);
+      ptx::mbar_wait(bar_w, 0, &never);
+    }
+  }
+  if (mma_issued && *abort_flag) {
+    int never = 0;
+    ptx::mbar_wait(bar_acc, 0, &never);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) ptx::tmem_dealloc(tmem, kRecN);
 }
 
 // ------------------------------------------------------------------ host side
@@ -366,42 +496,87 @@ int make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int b
   return THETA_OK;
 }
 
-template <int BN, int MODE>
-cudaError_t launch_tile_kernel(const LaunchCtx& c, const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& a2,
-                               const CUtensorMap& b2, const CUtensorMap& b3, const Args& args, int m_tiles,
-                               int n_tiles) {
-  using C = Cfg<BN, MODE>;
-  auto kern = umma_kernel<BN, MODE>;
-  static bool configured[64] = {};
-  if (!configured[c.device]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+// Per-device, per-kernel launch configuration: dynamic shared memory opt-in,
+// non-portable cluster sizes, and the number of co-resident CTAs per SM,
+// checked against tensor-memory capacity (co-resident CTAs must never need
+// more columns than an SM has, or allocation would stall).
+struct KernelInfo {
+  bool ready = false;
+  int blocks_per_sm = 0;
+  int max_cluster = 1;
+};
+
+template <typename Kern>
+cudaError_t prepare_kernel(KernelInfo* info, Kern kern, int threads, int smem, int tmem_cols, bool clusters) {
+  if (info->ready) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  if (clusters) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
-    int blocks = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, kThreads, C::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    // co-resident CTAs must never need more tensor memory than an SM has
-    if (blocks * C::kTmemCols > 512) return cudaErrorInvalidConfiguration;
-    configured[c.device] = true;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(n_tiles * args.splits), (unsigned)m_tiles, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = c.stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)args.splits;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a1, b1, a2, b2, b3, args);
+  int blocks = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, threads, smem);
+  if (e != cudaSuccess) return e;
+  if (blocks < 1 || blocks * tmem_cols > 512) return cudaErrorInvalidConfiguration;
+  info->blocks_per_sm = blocks;
+  info->max_cluster = 1;
+  if (clusters) {
+    // the largest cluster (16, else 8) that the GPU can place at all
+    for (int cs = 16; cs >= 8 && info->max_cluster == 1; cs /= 2) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(cs, 1, 1);
+      cfg.blockDim = dim3(threads, 1, 1);
+      cfg.dynamicSmemBytes = smem;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = cs;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) info->max_cluster = cs;
+    }
+    cudaGetLastError();  // a refused query above is not an error of this call
+    if (info->max_cluster == 1) return cudaErrorInvalidConfiguration;
+  }
+  info->ready = true;
+  return cudaSuccess;
 }
 
-int pick_splits(int64_t tiles, int kb, int num_sms) {
+// Largest power-of-two split (<= 16) that keeps every CTA resident in one
+// wave and leaves each split at least 4 K blocks.
+int pick_splits(int64_t tiles, int kb, int capacity, int max_cluster) {
   int s = 1;
-  while (s < 8 && tiles * s < 2 * (int64_t)num_sms && kb / (2 * s) >= 4) s *= 2;
+  while (2 * s <= max_cluster && tiles * (2 * s) <= capacity && kb / (2 * s) >= 4) s *= 2;
   return s;
+}
+
+template <int BN, int MODE>
+cudaError_t launch_tile_kernel(const LaunchCtx& c, const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& a2,
+                               const CUtensorMap& b2, const CUtensorMap& b3, Args args, int m_tiles, int n_tiles) {
+  using C = Cfg<BN, MODE>;
+  auto kern = umma_kernel<BN, MODE>;
+  static KernelInfo info[64];
+  cudaError_t e = prepare_kernel(&info[c.device], kern, kThreads, C::kSmemBytes, C::kTmemCols, true);
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = (int64_t)m_tiles * n_tiles;
+  args.splits = pick_splits(tiles, args.kb1, c.num_sms * info[c.device].blocks_per_sm, info[c.device].max_cluster);
+  return launch_pdl(kern, dim3((unsigned)(n_tiles * args.splits), (unsigned)m_tiles, 1), dim3(kThreads), C::kSmemBytes,
+                    c.stream, args.splits, a1, b1, a2, b2, b3, args);
+}
+
+template <int KB>
+cudaError_t launch_recon(const LaunchCtx& c, const CUtensorMap& mU, const CUtensorMap& mV, const CUtensorMap& mW0,
+                         const CUtensorMap& mOut, const float* s, int O, int I) {
+  using C = RecCfg<KB>;
+  auto kern = recon_kernel<KB>;
+  static KernelInfo info[64];
+  cudaError_t e = prepare_kernel(&info[c.device], kern, kRecThreads, C::kSmemBytes, kRecN, false);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3((unsigned)ceil_div(I, kRecN), (unsigned)ceil_div(O, kBM), 1), dim3(kRecThreads),
+                    C::kSmemBytes, c.stream, 1, mU, mV, mW0, mOut, s, O, I, c.err);
 }
 
 }  // namespace
@@ -415,18 +590,19 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
                         const void* V, int64_t M, int64_t O, int64_t I, int r, void* Y, void* ws,
                         cudaError_t* ce) {
   *ce = cudaSuccess;
-  if (O > (int64_t)65535 * kBM || M > (int64_t)1 << 30 || I > ((int64_t)1 << 31) - 64 || r > 256)
+  if (O > (int64_t)65535 * kBM || M > ((int64_t)1 << 30) || I > ((int64_t)1 << 31) - 64 || r > 256)
     return THETA_ERR_UNSUPPORTED;
   const int kb = (int)ceil_div(I, kBK);
   bf16* t_hi = nullptr;
   bf16* t_lo = nullptr;
   CUtensorMap mX, mW0, mU, mThi, mTlo, mV;
   int st;
-  if ((st = make_map(&mX, X, M, I, kBM, ce))) return st;  // XV A side (128 token rows)
+  cudaError_t e = cudaSuccess;
   if (r > 0) {
     t_hi = static_cast<bf16*>(ws);
     t_lo = reinterpret_cast<bf16*>(static_cast<uint8_t*>(ws) + forward_umma_workspace_bytes(M, r) / 2);
     // ---- T = X . V (fp32 in tensor memory) -> bf16 high and low parts
+    if ((st = make_map(&mX, X, M, I, kBM, ce))) return st;  // 128 token rows per tile
     if ((st = make_map(&mV, V, I, r, kBK, ce))) return st;  // box: 64 rank columns x 64 rows of I
     Args a = {};
     a.rows = (int)M;
@@ -438,9 +614,7 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
     a.r = r;
     a.err = c.err;
     const int m_tiles = (int)ceil_div(M, kBM);
-    a.splits = pick_splits(m_tiles, kb, c.num_sms);
     const int rp = (int)ceil_div(r, 64) * 64;
-    cudaError_t e;
     switch (rp) {
       case 64: e = launch_tile_kernel<64, MODE_XV>(c, mX, mV, mV, mV, mV, a, m_tiles, 1); break;
       case 128: e = launch_tile_kernel<128, MODE_XV>(c, mX, mV, mV, mV, mV, a, m_tiles, 1); break;
@@ -453,7 +627,7 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
     }
   }
   // ---- Y = s * (X . W0^T) + T . U^T, swap-AB: W0 rows are the MMA M side
-  const int BN = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  const int BN = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 256 ? 128 : 256;
   const int m_tiles = (int)ceil_div(O, kBM);
   const int n_tiles = (int)ceil_div(M, BN);
   if ((st = make_map(&mW0, W0, O, I, kBM, ce))) return st;
@@ -475,13 +649,12 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
   a.s = s;
   a.out = static_cast<bf16*>(Y);
   a.err = c.err;
-  a.splits = pick_splits((int64_t)m_tiles * n_tiles, kb, c.num_sms);
-  cudaError_t e;
   switch (BN) {
     case 16: e = launch_tile_kernel<16, MODE_FORWARD>(c, mW0, mXb, mU, mThi, mTlo, a, m_tiles, n_tiles); break;
     case 32: e = launch_tile_kernel<32, MODE_FORWARD>(c, mW0, mXb, mU, mThi, mTlo, a, m_tiles, n_tiles); break;
     case 64: e = launch_tile_kernel<64, MODE_FORWARD>(c, mW0, mXb, mU, mThi, mTlo, a, m_tiles, n_tiles); break;
-    default: e = launch_tile_kernel<128, MODE_FORWARD>(c, mW0, mXb, mU, mThi, mTlo, a, m_tiles, n_tiles); break;
+    case 128: e = launch_tile_kernel<128, MODE_FORWARD>(c, mW0, mXb, mU, mThi, mTlo, a, m_tiles, n_tiles); break;
+    default: e = launch_tile_kernel<256, MODE_FORWARD>(c, mW0, mXb, mU, mThi, mTlo, a, m_tiles, n_tiles); break;
   }
   if (e != cudaSuccess) {
     *ce = e;
@@ -497,29 +670,25 @@ int launch_reconstruct_umma(const LaunchCtx& c, const float* s, const void* W0, 
     const int64_t nvec = O * I / 8;
     int64_t grid = ceil_div(nvec, 256);
     if (grid > 8 * (int64_t)c.num_sms) grid = 8 * (int64_t)c.num_sms;
-    scale_rows_kernel<<<(unsigned)grid, 256, 0, c.stream>>>(s, static_cast<const bf16*>(W0), I, nvec,
-                                                           static_cast<bf16*>(W_out));
-    *ce = cudaGetLastError();
+    if (grid < 1) grid = 1;
+    *ce = launch_pdl(scale_rows_kernel, dim3((unsigned)grid), dim3(256), 0, c.stream, 1, s,
+                     static_cast<const bf16*>(W0), I, nvec, static_cast<bf16*>(W_out));
     return *ce == cudaSuccess ? THETA_OK : THETA_ERR_CUDA;
   }
-  if (O > (int64_t)65535 * kBM || I > ((int64_t)1 << 31) - 256 || r > ((int64_t)1 << 20)) return THETA_ERR_UNSUPPORTED;
-  constexpr int BN = 128;
-  CUtensorMap mU, mV;
+  if (O > (int64_t)65535 * kBM || I > ((int64_t)1 << 31) - 256 || r > 256) return THETA_ERR_UNSUPPORTED;
+  CUtensorMap mU, mV, mW0, mOut;
   int st;
   if ((st = make_map(&mU, U, O, r, kBM, ce))) return st;
-  if ((st = make_map(&mV, V, I, r, BN, ce))) return st;
-  Args a = {};
-  a.rows = (int)O;
-  a.cols = (int)I;
-  a.kb1 = (int)ceil_div(r, kBK);
-  a.kb2 = 0;
-  a.splits = 1;
-  a.s = s;
-  a.W0 = static_cast<const bf16*>(W0);
-  a.out = static_cast<bf16*>(W_out);
-  a.err = c.err;
-  cudaError_t e = launch_tile_kernel<BN, MODE_RECON>(c, mU, mV, mU, mV, mV, a, (int)ceil_div(O, kBM),
-                                                     (int)ceil_div(I, BN));
+  if ((st = make_map(&mV, V, I, r, kRecN, ce))) return st;
+  if ((st = make_map(&mW0, W0, O, I, kBM, ce))) return st;
+  if ((st = make_map(&mOut, W_out, O, I, kBM, ce))) return st;
+  cudaError_t e;
+  switch ((int)ceil_div(r, kBK)) {
+    case 1: e = launch_recon<1>(c, mU, mV, mW0, mOut, s, (int)O, (int)I); break;
+    case 2: e = launch_recon<2>(c, mU, mV, mW0, mOut, s, (int)O, (int)I); break;
+    case 3: e = launch_recon<3>(c, mU, mV, mW0, mOut, s, (int)O, (int)I); break;
+    default: e = launch_recon<4>(c, mU, mV, mW0, mOut, s, (int)O, (int)I); break;
+  }
   if (e != cudaSuccess) {
     *ce = e;
     return THETA_ERR_CUDA;

@@ -61,6 +61,11 @@ FORWARD_CASES = [
     (300, 392, 328, 64),
     (1, 8, 8, 8),
     (5, 2056, 200, 8),
+    (600, 256, 1152, 32),    # three 256-token tiles
+    (40, 256, 264, 128),     # rank variants of the T = X.V kernel
+    (8, 136, 200, 192),
+    (130, 264, 392, 256),
+    (3, 1024, 6912, 16),     # deep K: split across a cluster
 ]
 
 
@@ -104,7 +109,7 @@ def test_forward_equals_rebuilt_weight_projection(lib, torch, dt):
 
 # ---------------------------------------------------------------- reconstruct
 RECON_CASES = [(256, 256, 8), (392, 328, 32), (136, 1160, 64), (1024, 1152, 32), (40, 24, 0), (8, 8, 8),
-               (2056, 200, 24)]
+               (2056, 200, 24), (200, 136, 128), (64, 520, 192), (72, 264, 256), (128, 64, 64)]
 
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
