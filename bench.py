@@ -55,13 +55,10 @@ BF16 = 2  # bytes
 
 
 # --------------------------------------------------------------- accounting
-def bytes_band_mean(L, G, O, I, b=BF16):
-    return L * O * I * b + G * O * I * b
-
-
-def bytes_rowscale_residual(L, G, O, I, b=BF16):
-    # read every W once and each band's W0 once; write s (fp32) and R
-    return L * O * I * b + G * O * I * b + 4 * L * O + L * O * I * b
+def bytes_prelude(L, G, O, I, b=BF16):
+    """Minimum traffic of the whole prelude of one family: read every W once,
+    write the G shared blocks, the L residuals and the L fp32 scales."""
+    return L * O * I * b + G * O * I * b + L * O * I * b + 4 * L * O
 
 
 def bytes_reconstruct(O, I, r, b=BF16):
@@ -88,14 +85,16 @@ def step_accounting(model=MODEL, r=RANK, m_values=M_VALUES, g_values=G_VALUES):
         pre = rec = fro = 0
         fwd = {m: [0, 0] for m in m_values}
         for fam, (O, I) in model.shapes.items():
-            pre += bytes_band_mean(L, G, O, I) + bytes_rowscale_residual(L, G, O, I)
+            pre += bytes_prelude(L, G, O, I)
             rec += L * bytes_reconstruct(O, I, r)
             fro += L * bytes_frob(O, I)
             for m in m_values:
                 fwd[m][0] += L * bytes_forward(m, O, I, r)
                 fwd[m][1] += L * flops_forward(m, O, I, r)
         nf = len(model.shapes)
-        stages.append(dict(name=f"prelude_G{G}", kind="prelude", bytes=pre, flops=0, launches=nf * G * 2))
+        fused = L // G <= 4  # bands of <= 4 layers run as one kernel per band
+        stages.append(dict(name=f"prelude_G{G}", kind="prelude", bytes=pre, flops=0,
+                           launches=nf * G * (1 if fused else 2)))
         stages.append(dict(name=f"reconstruct_G{G}", kind="reconstruct", bytes=rec, flops=0, launches=nf * L))
         stages.append(dict(name=f"frob_G{G}", kind="frob", bytes=fro, flops=0, launches=nf * L * 2))
         for m in m_values:
@@ -334,7 +333,7 @@ def oracle_sample_step(rows=64, seed=0, model=MODEL, r=RANK):
                 oracle.frob_error(w[l], rec)
                 for m in M_VALUES:
                     oracle.linear_forward(X[m], w0, s32, U[l], V[l], "bf16")
-            total_bytes += bytes_band_mean(L, G, n, I) + bytes_rowscale_residual(L, G, n, I)
+            total_bytes += bytes_prelude(L, G, n, I)
             total_bytes += L * (bytes_reconstruct(n, I, r) + bytes_frob(n, I))
             total_bytes += L * sum(bytes_forward(m, n, I, r) for m in M_VALUES)
     return total_bytes, time.perf_counter() - t0
@@ -585,9 +584,9 @@ def run_op(args):
         W = syn.device_family_weights(L, O, I, seed=seed, family="op")
         W0 = [torch.empty(O, I, dtype=torch.bfloat16, device="cuda") for _ in range(G)]
         sl = [torch.empty(O, dtype=torch.float32, device="cuda") for _ in range(L)]
-        R = [torch.empty(O, I, dtype=torch.bfloat16, device="cuda") for _ in range(L)]
+        R = None if args.no_residual else [torch.empty(O, I, dtype=torch.bfloat16, device="cuda") for _ in range(L)]
         call = lambda: theta.theta_decompose_prelude(W, G, W0, sl, R)  # noqa: E731
-        nbytes, nflops = bytes_band_mean(L, G, O, I) + bytes_rowscale_residual(L, G, O, I), 0
+        nbytes, nflops = bytes_prelude(L, G, O, I) - (L * O * I * BF16 if args.no_residual else 0), 0
     elif args.op == "frob":
         A = syn.device_normal((O, I), 0.02, seed, "A", O, I)
         B = syn.device_normal((O, I), 0.02, seed, "B", O, I)
@@ -646,6 +645,7 @@ def main(argv=None):
     ap.add_argument("--layers", type=int, default=4)
     ap.add_argument("--G", type=int, default=1)
     ap.add_argument("--iters", type=int, default=20)
+    ap.add_argument("--no-residual", action="store_true", help="--op prelude: skip the residual output")
     args = ap.parse_args(argv)
     if args.op:
         return run_op(args)

@@ -23,10 +23,6 @@ __all__ = [
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtheta.so")
-if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m linear_theta_forward_b200.build`")
-
-lib = ctypes.CDLL(LIB_PATH)
 
 THETA_F32, THETA_BF16 = 0, 1
 THETA_OP_FROB_ERROR, THETA_OP_LINEAR_FORWARD = 0, 1
@@ -38,36 +34,52 @@ _i64 = ctypes.c_int64
 _int = ctypes.c_int
 _sz = ctypes.c_size_t
 
+_SIGNATURES = {
+    "theta_version": (_int,),
+    "theta_status_string": (ctypes.c_char_p, _int),
+    "theta_last_error": (ctypes.c_char_p,),
+    "theta_band_index": (_int, _int, _int, _i32p, _i32p),
+    "theta_band_mean": (_int, _vp, _int, _i64, _i64, _int, _vp, _vp),
+    "theta_row_scale": (_int, _vp, _vp, _i64, _i64, _int, _vp, _vp),
+    "theta_residual": (_int, _vp, _vp, _vp, _i64, _i64, _int, _vp, _vp),
+    "theta_decompose_prelude": (_int, _vp, _int, _int, _i64, _i64, _int, _vp, _vp, _vp, _vp),
+    "theta_reconstruct": (_int, _vp, _vp, _vp, _vp, _i64, _i64, _int, _int, _vp, _vp),
+    "theta_frob_error": (_int, _vp, _vp, _i64, _int, _vp, _vp, _sz, _vp),
+    "theta_linear_forward": (_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp, _sz, _vp),
+    "theta_linear_forward_noalloc": (_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp),
+    "theta_workspace_size": (_int, _int, _i64, _i64, _i64, _int, _int, ctypes.POINTER(_sz)),
+    "theta_device_status": (_int, _vp),
+}
 
-def _sig(name, res, *args):
-    f = getattr(lib, name)
-    f.restype = res
-    f.argtypes = list(args)
-    return f
+_LIB = None
 
 
-_sig("theta_version", _int)
-_sig("theta_status_string", ctypes.c_char_p, _int)
-_sig("theta_last_error", ctypes.c_char_p)
-_sig("theta_band_index", _int, _int, _int, _i32p, _i32p)
-_sig("theta_band_mean", _int, _vp, _int, _i64, _i64, _int, _vp, _vp)
-_sig("theta_row_scale", _int, _vp, _vp, _i64, _i64, _int, _vp, _vp)
-_sig("theta_residual", _int, _vp, _vp, _vp, _i64, _i64, _int, _vp, _vp)
-_sig("theta_decompose_prelude", _int, _vp, _int, _int, _i64, _i64, _int, _vp, _vp, _vp, _vp)
-_sig("theta_reconstruct", _int, _vp, _vp, _vp, _vp, _i64, _i64, _int, _int, _vp, _vp)
-_sig("theta_frob_error", _int, _vp, _vp, _i64, _int, _vp, _vp, _sz, _vp)
-_sig("theta_linear_forward", _int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp,
-     _sz, _vp)
-_sig("theta_linear_forward_noalloc", _int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp)
-_sig("theta_workspace_size", _int, _int, _i64, _i64, _i64, _int, _int, ctypes.POINTER(_sz))
-_sig("theta_device_status", _int, _vp)
+def _load():
+    """The loaded libtheta.so (loaded on first use; a missing build is an error)."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m linear_theta_forward_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, *args) in _SIGNATURES.items():
+            f = getattr(handle, name)
+            f.restype = res
+            f.argtypes = list(args)
+        _LIB = handle
+    return _LIB
+
+
+def __getattr__(name):
+    if name == "lib":
+        return _load()
+    raise AttributeError(name)
 
 
 class ThetaError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        msg = lib.theta_last_error().decode(errors="replace")
-        name = lib.theta_status_string(status).decode()
+        msg = _load().theta_last_error().decode(errors="replace")
+        name = _load().theta_status_string(status).decode()
         super().__init__(f"{where}: {name} ({status}): {msg}")
 
 
@@ -121,31 +133,31 @@ def _ptr_array(tensors, name):
 
 # ------------------------------------------------------------------ host-only
 def theta_version() -> int:
-    return lib.theta_version()
+    return _load().theta_version()
 
 
 def theta_status_string(status: int) -> str:
-    return lib.theta_status_string(status).decode()
+    return _load().theta_status_string(status).decode()
 
 
 def theta_last_error() -> str:
-    return lib.theta_last_error().decode(errors="replace")
+    return _load().theta_last_error().decode(errors="replace")
 
 
 def theta_band_index(num_layers: int, G: int):
     """(band_of_layer int32[num_layers], band_start int32[G + 1])."""
     if num_layers < 1:
-        _check(lib.theta_band_index(num_layers, G, None, None), "theta_band_index")
+        _check(_load().theta_band_index(num_layers, G, None, None), "theta_band_index")
     bol = np.zeros(num_layers, dtype=np.int32)
     start = np.zeros(max(G, 0) + 1, dtype=np.int32)
-    _check(lib.theta_band_index(num_layers, G, bol.ctypes.data_as(_i32p), start.ctypes.data_as(_i32p)),
+    _check(_load().theta_band_index(num_layers, G, bol.ctypes.data_as(_i32p), start.ctypes.data_as(_i32p)),
            "theta_band_index")
     return bol, start
 
 
 def theta_workspace_size(op: int, M: int, O: int, I: int, rank: int, dtype) -> int:
     out = _sz(0)
-    _check(lib.theta_workspace_size(op, M, O, I, rank, _dtype_of(dtype), ctypes.byref(out)),
+    _check(_load().theta_workspace_size(op, M, O, I, rank, _dtype_of(dtype), ctypes.byref(out)),
            "theta_workspace_size")
     return out.value
 
@@ -154,19 +166,19 @@ def theta_workspace_size(op: int, M: int, O: int, I: int, rank: int, dtype) -> i
 def theta_band_mean(weights, W0, stream=None) -> None:
     O, I = W0.shape
     arr = _ptr_array(weights, "weights")
-    _check(lib.theta_band_mean(ctypes.cast(arr, _vp), len(weights), O, I, _dtype_code(W0),
+    _check(_load().theta_band_mean(ctypes.cast(arr, _vp), len(weights), O, I, _dtype_code(W0),
                                _ptr(W0, "W0"), _stream(stream)), "theta_band_mean")
 
 
 def theta_row_scale(weight, W0, s, stream=None) -> None:
     O, I = W0.shape
-    _check(lib.theta_row_scale(_ptr(weight, "weight"), _ptr(W0, "W0"), O, I, _dtype_code(W0),
+    _check(_load().theta_row_scale(_ptr(weight, "weight"), _ptr(W0, "W0"), O, I, _dtype_code(W0),
                                _ptr(s, "s"), _stream(stream)), "theta_row_scale")
 
 
 def theta_residual(weight, W0, s, R, stream=None) -> None:
     O, I = W0.shape
-    _check(lib.theta_residual(_ptr(weight, "weight"), _ptr(W0, "W0"), _ptr(s, "s"), O, I,
+    _check(_load().theta_residual(_ptr(weight, "weight"), _ptr(W0, "W0"), _ptr(s, "s"), O, I,
                               _dtype_code(W0), _ptr(R, "R"), _stream(stream)), "theta_residual")
 
 
@@ -178,7 +190,7 @@ def theta_decompose_prelude(weights, G: int, W0, s, residual=None, stream=None) 
     w0 = _ptr_array(W0, "W0")
     sp = _ptr_array(s, "s")
     rp = _ptr_array(residual, "residual") if residual is not None else None
-    _check(lib.theta_decompose_prelude(ctypes.cast(w, _vp), len(weights), G, O, I,
+    _check(_load().theta_decompose_prelude(ctypes.cast(w, _vp), len(weights), G, O, I,
                                        _dtype_code(weights[0]), ctypes.cast(w0, _vp),
                                        ctypes.cast(sp, _vp),
                                        ctypes.cast(rp, _vp) if rp is not None else None,
@@ -188,7 +200,7 @@ def theta_decompose_prelude(weights, G: int, W0, s, residual=None, stream=None) 
 def theta_reconstruct(s, W0, U, V, W_out, stream=None) -> None:
     O, I = W0.shape
     rank = 0 if U is None else U.shape[1]
-    _check(lib.theta_reconstruct(_ptr(s, "s"), _ptr(W0, "W0"), _ptr(U, "U", optional=True),
+    _check(_load().theta_reconstruct(_ptr(s, "s"), _ptr(W0, "W0"), _ptr(U, "U", optional=True),
                                  _ptr(V, "V", optional=True), O, I, rank, _dtype_code(W0),
                                  _ptr(W_out, "W_out"), _stream(stream)), "theta_reconstruct")
 
@@ -196,7 +208,7 @@ def theta_reconstruct(s, W0, U, V, W_out, stream=None) -> None:
 def theta_frob_error(original, reconstructed, out, workspace, stream=None) -> None:
     """out: float64 CUDA tensor of one element; workspace: CUDA tensor of at
     least theta_workspace_size(THETA_OP_FROB_ERROR, ...) bytes."""
-    _check(lib.theta_frob_error(_ptr(original, "original"), _ptr(reconstructed, "reconstructed"),
+    _check(_load().theta_frob_error(_ptr(original, "original"), _ptr(reconstructed, "reconstructed"),
                                 original.numel(), _dtype_code(original), _ptr(out, "out"),
                                 _ptr(workspace, "workspace"),
                                 workspace.numel() * workspace.element_size(), _stream(stream)),
@@ -211,7 +223,7 @@ def theta_linear_forward(X, W0, s, U, V, Y, workspace=None, stream=None) -> None
     rank = 0 if U is None else U.shape[1]
     ws_ptr = _ptr(workspace, "workspace", optional=True)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    _check(lib.theta_linear_forward(_ptr(X, "X"), M, I, _ptr(W0, "W0"), O, _ptr(s, "s"),
+    _check(_load().theta_linear_forward(_ptr(X, "X"), M, I, _ptr(W0, "W0"), O, _ptr(s, "s"),
                                     _ptr(U, "U", optional=True), _ptr(V, "V", optional=True), rank,
                                     _dtype_code(X), _ptr(Y, "Y"), ws_ptr, ws_bytes, _stream(stream)),
            "theta_linear_forward")
@@ -224,11 +236,11 @@ def theta_linear_forward_noalloc(X, W0, s, U, V, Y, stream=None) -> None:
     M, I = X.shape
     O = W0.shape[0]
     rank = 0 if U is None else U.shape[1]
-    _check(lib.theta_linear_forward_noalloc(_ptr(X, "X"), M, I, _ptr(W0, "W0"), O, _ptr(s, "s"),
+    _check(_load().theta_linear_forward_noalloc(_ptr(X, "X"), M, I, _ptr(W0, "W0"), O, _ptr(s, "s"),
                                             _ptr(U, "U", optional=True), _ptr(V, "V", optional=True), rank,
                                             _dtype_code(X), _ptr(Y, "Y"), _stream(stream)),
            "theta_linear_forward_noalloc")
 
 
 def theta_device_status(stream=None) -> None:
-    _check(lib.theta_device_status(_stream(stream)), "theta_device_status")
+    _check(_load().theta_device_status(_stream(stream)), "theta_device_status")

@@ -22,7 +22,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libtheta.so")
 
-SOURCES = ["theta_api.cu", "stream_kernels.cu", "simt_kernels.cu", "umma_kernels.cu", "noalloc.cu"]
+SOURCES = ["theta_api.cu", "stream_kernels.cu", "prelude_kernels.cu", "simt_kernels.cu", "umma_kernels.cu",
+           "noalloc.cu"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + [

@@ -25,6 +25,13 @@ cudaError_t launch_rowscale_band(const LaunchCtx& c, theta_dtype dt, const void*
                                  float* const* s, void* const* R);
 cudaError_t launch_residual(const LaunchCtx& c, theta_dtype dt, const void* w, const void* W0,
                             const float* s, int64_t O, int64_t I, void* R);
+// ---- prelude pipeline (prelude_kernels.cu): every band of a family in one
+// launch. band_mode: bands of <= 4 layers, forms W0, s and R in one pass;
+// otherwise reads the already-formed W0 and writes s and R. Returns false
+// without launching when the problem does not fit the pipeline.
+bool launch_prelude_pipe(const LaunchCtx& c, theta_dtype dt, bool band_mode, const void* const* w, int L, int G,
+                         const int32_t* band_start, const int32_t* band_of_layer, void* const* W0,
+                         float* const* s, void* const* R, int64_t O, int64_t I, cudaError_t* e);
 size_t frob_workspace_bytes();
 cudaError_t launch_frob(const LaunchCtx& c, theta_dtype dt, const void* a, const void* b,
                         int64_t n, double* out, void* ws);

@@ -355,6 +355,23 @@ int round_vpt(int64_t v) {
   return -1;
 }
 
+// Ring geometry for `rows_per_item` rows of I elements per slot: up to 16
+// slots within ~100 KB (two CTAs per SM), at least 2 slots; 0 if it does not fit.
+// Threads per row and vectors per thread for a row of nv vectors: the
+// fewest threads that keep every thread at <= 4 vectors, else 256 threads.
+void row_geometry(int64_t nv, int* tpr, int* vpt) {
+  *tpr = 0;
+  const int tprs[] = {32, 64, 128, 256};
+  for (int cand : tprs) {
+    if (ceil_div(nv, cand) <= 4) {
+      *tpr = cand;
+      break;
+    }
+  }
+  if (!*tpr) *tpr = 256;
+  *vpt = round_vpt(ceil_div(nv, *tpr));
+}
+
 template <typename T>
 cudaError_t rowscale_t(const LaunchCtx& c, const void* W0, const void* const* w, int n, int64_t O,
                        int64_t I, float* const* s, void* const* R) {
@@ -368,19 +385,9 @@ cudaError_t rowscale_t(const LaunchCtx& c, const void* W0, const void* const* w,
     rt.p[l] = write_r ? R[l] : nullptr;
     ok = ok && aligned16(w[l]) && (!write_r || aligned16(R[l]));
   }
-  const int64_t nv = I / Vec<T>::N;
+
   int tpr = 0, vpt = -1;
-  if (ok) {
-    const int tprs[] = {32, 64, 128, 256};
-    for (int cand : tprs) {
-      if (ceil_div(nv, cand) <= 4) {
-        tpr = cand;
-        break;
-      }
-    }
-    if (!tpr) tpr = 256;
-    vpt = round_vpt(ceil_div(nv, tpr));
-  }
+  if (ok) row_geometry(I / Vec<T>::N, &tpr, &vpt);
   if (vpt > 0) {
     const int groups = kThreads / tpr;
     const int grid = grid_for(c, O, groups, vpt <= 4 ? 8 : 4);

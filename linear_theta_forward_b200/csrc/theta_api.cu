@@ -158,6 +158,13 @@ THETA_API int theta_row_scale(const void* weight, const void* W0, int64_t O, int
   if (st) return st;
   const void* w[1] = {weight};
   float* sp[1] = {s};
+  void* w0[1] = {const_cast<void*>(W0)};
+  const int32_t band_start[2] = {0, 1}, band_of_layer[1] = {0};
+  cudaError_t pe = cudaSuccess;
+  if (launch_prelude_pipe(c, dt, false, w, 1, 1, band_start, band_of_layer, w0, sp, nullptr, O, I, &pe)) {
+    CHECK_LAUNCH(pe, "theta_row_scale launch");
+    return THETA_OK;
+  }
   CHECK_LAUNCH(launch_rowscale_band(c, dt, W0, w, 1, O, I, sp, nullptr), "theta_row_scale launch");
   return THETA_OK;
 }
@@ -194,9 +201,25 @@ THETA_API int theta_decompose_prelude(const void* const* weights, int num_layers
   if (st) return st;
   int32_t band_of_layer[THETA_MAX_LAYERS], band_start[THETA_MAX_LAYERS + 1];
   theta_band_index(num_layers, G, band_of_layer, band_start);
+  const int nmax = (num_layers + G - 1) / G;
+  cudaError_t pe = cudaSuccess;
+  // bands of <= 4 layers: one pass over the family forms W0, s and R
+  if (nmax <= 4 && launch_prelude_pipe(c, dt, true, weights, num_layers, G, band_start, band_of_layer, W0, s,
+                                       residual, O, I, &pe)) {
+    CHECK_LAUNCH(pe, "prelude launch");
+    return THETA_OK;
+  }
   for (int b = 0; b < G; ++b) {
     const int first = band_start[b], n = band_start[b + 1] - band_start[b];
     CHECK_LAUNCH(launch_band_mean(c, dt, weights + first, n, O, I, W0[b]), "band mean launch");
+  }
+  if (launch_prelude_pipe(c, dt, false, weights, num_layers, G, band_start, band_of_layer, W0, s, residual, O, I,
+                          &pe)) {
+    CHECK_LAUNCH(pe, "row scale launch");
+    return THETA_OK;
+  }
+  for (int b = 0; b < G; ++b) {
+    const int first = band_start[b], n = band_start[b + 1] - band_start[b];
     CHECK_LAUNCH(launch_rowscale_band(c, dt, W0[b], weights + first, n, O, I, s + first,
                                       residual ? residual + first : nullptr),
                  "row scale launch");

@@ -60,6 +60,7 @@ struct Args {
   bf16* t_hi;      // XV outputs [rows, r]
   bf16* t_lo;
   int r;
+  int early_start;  // FORWARD after its own T = X.V kernel: see the producer
   unsigned* err;
 };
 
@@ -121,7 +122,15 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_enter();
+  // Programmatic dependent launch. Normally every thread waits here for the
+  // previous grid before touching global memory. A forward launched right
+  // after its own T = X.V kernel starts early instead: that kernel waited for
+  // all earlier work before it let this grid launch, and it writes only T, so
+  // W0, X and s may be streamed at once; only the loads of T (the producer's
+  // rank phase) and the epilogue wait.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const bool early = MODE == MODE_FORWARD && args.early_start;
+  if (!early) asm volatile("griddepcontrol.wait;" ::: "memory");
 
   auto give_up = [&]() {
     record_timeout(args.err);
@@ -156,6 +165,7 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
         }
       } else {
         const int j = i - n1;
+        if (early && j == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
         const int jx = (j % args.kb2) * kBK;
         ptx::tma_load_2d(a, &tmA2, &full[st], jx, m_tile * kBM);
         ptx::tma_load_2d(b, j < args.kb2 ? &tmB2 : &tmB3, &full[st], jx, n_tile * BN);
@@ -219,6 +229,7 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;  // accumulator row = TMEM lane
     const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
+    if (early) asm volatile("griddepcontrol.wait;" ::: "memory");
     bool ok = ptx::mbar_wait(accum, 0, abort_flag);
     if (!ok) give_up();
     ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
@@ -511,6 +522,10 @@ cudaError_t prepare_kernel(KernelInfo* info, Kern kern, int threads, int smem, i
   if (info->ready) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  // all of the unified L1/shared array as shared memory: the stage rings are
+  // what keeps loads in flight, and the residency count below relies on it
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e != cudaSuccess) return e;
   if (clusters) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
@@ -648,6 +663,7 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
   a.kb2 = r > 0 ? (int)ceil_div(r, kBK) : 0;
   a.s = s;
   a.out = static_cast<bf16*>(Y);
+  a.early_start = r > 0;  // directly after this call's T = X.V kernel
   a.err = c.err;
   switch (BN) {
     case 16: e = launch_tile_kernel<16, MODE_FORWARD>(c, mW0, mXb, mU, mThi, mTlo, a, m_tiles, n_tiles); break;

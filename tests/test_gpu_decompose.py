@@ -96,7 +96,10 @@ def test_zero_w0_row_gives_zero_scale(lib, torch):
                                         ("bf16", 7, 3, 40, 264),
                                         ("bf16", 26, 4, 24, 1152),
                                         ("f32", 5, 2, 17, 13),
-                                        ("bf16", 6, 1, 9, 5376)])
+                                        ("bf16", 6, 1, 9, 5376),
+                                        ("bf16", 8, 2, 33, 5376),     # one-pass prelude, 4-layer bands
+                                        ("bf16", 2, 2, 20, 21504),    # one-pass prelude, widest rows
+                                        ("f32", 3, 1, 21, 1000)])
 def test_decompose_prelude(lib, torch, dt, L, G, O, I):
     w = weights(L, O, I, dt, seed=L * G)
     ws = [dev(w[i], dt) for i in range(L)]
