@@ -93,6 +93,17 @@ __device__ __forceinline__ R ld_stream(const R* p) {
   return __ldg(p);
 }
 
+// x / n rounded once (IEEE division). For n a power of two the quotient is
+// x * 2^-k, which is what the multiplication below computes and rounds
+// identically, so the costly division sequence runs only for other n.
+struct DivByCount {
+  float inv;
+  float fn;
+  bool pow2;
+  __device__ __forceinline__ explicit DivByCount(int n) : inv(1.f / (float)n), fn((float)n), pow2((n & (n - 1)) == 0) {}
+  __device__ __forceinline__ float operator()(float x) const { return pow2 ? x * inv : __fdiv_rn(x, fn); }
+};
+
 // ------------------------------------------------------------- reductions
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll

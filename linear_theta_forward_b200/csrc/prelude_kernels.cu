@@ -165,6 +165,7 @@ prelude_pipe_kernel(const __grid_constant__ PreludeArgs a) {
         n = a.band_start[bl + 1] - first;
       }
       const uint8_t* rowp = ring + (size_t)st * a.slot_bytes + g * row_stride;
+      const DivByCount div_n(n);
       // W0 row (registers); BAND forms it from the band's rows and writes it
       R w0[VPT];
 #pragma unroll
@@ -175,6 +176,11 @@ prelude_pipe_kernel(const __grid_constant__ PreludeArgs a) {
           continue;
         }
         if constexpr (BAND) {
+          if (n == 1) {  // the shared block of a one-layer band is that layer
+            w0[q] = reinterpret_cast<const R*>(rowp)[v];
+            reinterpret_cast<R*>(static_cast<T*>(a.W0.p[bl]) + o * a.I)[v] = w0[q];
+            continue;
+          }
           float acc[V::N];
 #pragma unroll
           for (int e = 0; e < V::N; ++e) acc[e] = 0.f;
@@ -187,9 +193,8 @@ prelude_pipe_kernel(const __grid_constant__ PreludeArgs a) {
               for (int e = 0; e < V::N; ++e) acc[e] += f[e];
             }
           }
-          const float fn = (float)n;
 #pragma unroll
-          for (int e = 0; e < V::N; ++e) acc[e] = __fdiv_rn(acc[e], fn);
+          for (int e = 0; e < V::N; ++e) acc[e] = div_n(acc[e]);
           w0[q] = pack(acc, (R*)nullptr);
           reinterpret_cast<R*>(static_cast<T*>(a.W0.p[bl]) + o * a.I)[v] = w0[q];
         } else {
@@ -264,20 +269,25 @@ prelude_pipe_kernel(const __grid_constant__ PreludeArgs a) {
   }
 }
 
-// Threads per row: the fewest (32..256) that keep each thread at <= 4
-// vectors of the row, else 256; vectors per thread rounded up to a variant.
-bool geometry(int64_t nv, int* tpr, int* vpt) {
+// Threads per output row (32..256, i.e. 8..1 rows per item): the fewest
+// that keep each thread at <= 12 vectors of a row and an item's shared
+// memory within 32 KB, so a CTA has several items in flight and each item
+// carries enough bytes to pay for its one reduction barrier. Vectors per
+// thread are rounded up to a compiled variant.
+bool geometry(int64_t nv, int64_t per_row_bytes, int* tpr, int* vpt) {
   const int tprs[] = {32, 64, 128, 256};
-  *tpr = 256;
-  for (int c : tprs)
-    if (ceil_div(nv, c) <= 4) {
+  *tpr = 0;
+  for (int c : tprs) {
+    if (ceil_div(nv, c) <= 12 && (kConsumers / c) * per_row_bytes <= 32 * 1024) {
       *tpr = c;
       break;
     }
+  }
+  if (!*tpr) *tpr = 256;
   const int64_t need = ceil_div(nv, *tpr);
   const int opts[] = {1, 2, 3, 4, 6, 8, 12};
   for (int o : opts)
-    if (need <= o && (o <= 4 || *tpr == 256)) {
+    if (need <= o) {
       *vpt = o;
       return true;
     }
@@ -304,13 +314,9 @@ cudaError_t dispatch_vpt(const LaunchCtx& c, const PreludeArgs& a, int vpt, int 
     case 2: return launch_one<T, BAND, TPR, 2>(c, a, grid, smem);
     case 3: return launch_one<T, BAND, TPR, 3>(c, a, grid, smem);
     case 4: return launch_one<T, BAND, TPR, 4>(c, a, grid, smem);
-  }
-  if constexpr (TPR == 256) {
-    switch (vpt) {
-      case 6: return launch_one<T, BAND, TPR, 6>(c, a, grid, smem);
-      case 8: return launch_one<T, BAND, TPR, 8>(c, a, grid, smem);
-      case 12: return launch_one<T, BAND, TPR, 12>(c, a, grid, smem);
-    }
+    case 6: return launch_one<T, BAND, TPR, 6>(c, a, grid, smem);
+    case 8: return launch_one<T, BAND, TPR, 8>(c, a, grid, smem);
+    case 12: return launch_one<T, BAND, TPR, 12>(c, a, grid, smem);
   }
   return cudaErrorInvalidValue;
 }
@@ -324,13 +330,13 @@ bool plan(const LaunchCtx& c, const void* const* w, int L, int G, const int32_t*
           const int32_t* band_of_layer, void* const* W0, float* const* s, void* const* R, int64_t O, int64_t I,
           PreludeArgs* a, int* tpr, int* vpt, int* grid, size_t* smem) {
   if (I % Vec<T>::N) return false;
-  if (!geometry(I / Vec<T>::N, tpr, vpt)) return false;
-  const int rows = kConsumers / *tpr;
   int nmax = 1;
   for (int b = 0; b < G; ++b) nmax = max(nmax, band_start[b + 1] - band_start[b]);
   if (BAND && nmax > 4) return false;
   const int64_t row_bytes = I * (int64_t)sizeof(T);
   const int64_t per_row = BAND ? nmax * row_bytes : 2 * row_bytes;
+  if (!geometry(I / Vec<T>::N, per_row, tpr, vpt)) return false;
+  const int rows = kConsumers / *tpr;
   const int64_t slot = ceil_div(rows * per_row, 128) * 128;
   int64_t slots = kSmemBudget / slot;
   if (slots > kMaxSlots) slots = kMaxSlots;

@@ -37,7 +37,7 @@ band_mean_kernel(PtrTable src, int n, int64_t nvec, int64_t count, T* __restrict
   pdl_enter();
   using V = Vec<T>;
   using R = typename V::raw;
-  const float fn = (float)n;
+  const DivByCount div_n(n);
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   for (int64_t v = tid; v < nvec; v += stride) {
@@ -64,14 +64,14 @@ band_mean_kernel(PtrTable src, int n, int64_t nvec, int64_t count, T* __restrict
       for (int e = 0; e < V::N; ++e) acc[e] += f[e];
     }
 #pragma unroll
-    for (int e = 0; e < V::N; ++e) acc[e] = __fdiv_rn(acc[e], fn);
+    for (int e = 0; e < V::N; ++e) acc[e] = div_n(acc[e]);
     reinterpret_cast<R*>(out)[v] = pack(acc, (R*)nullptr);
   }
   // scalar tail (count not a multiple of the vector width)
   for (int64_t i = nvec * V::N + tid; i < count; i += stride) {
     float acc = 0.f;
     for (int l = 0; l < n; ++l) acc += to_f32(static_cast<const T*>(src.p[l])[i]);
-    out[i] = from_f32<T>(__fdiv_rn(acc, fn));
+    out[i] = from_f32<T>(div_n(acc));
   }
 }
 
