@@ -92,9 +92,11 @@ def step_accounting(model=MODEL, r=RANK, m_values=M_VALUES, g_values=G_VALUES):
                 fwd[m][0] += L * bytes_forward(m, O, I, r)
                 fwd[m][1] += L * flops_forward(m, O, I, r)
         nf = len(model.shapes)
-        fused = L // G <= 4  # bands of <= 4 layers run as one kernel per band
+        # bands of <= 4 layers: one pipeline launch per family forms W0, s and R;
+        # longer bands: one band-mean launch per band, then one pipeline launch
+        one_pass = -(-L // G) <= 4
         stages.append(dict(name=f"prelude_G{G}", kind="prelude", bytes=pre, flops=0,
-                           launches=nf * G * (1 if fused else 2)))
+                           launches=nf * (1 if one_pass else G + 1)))
         stages.append(dict(name=f"reconstruct_G{G}", kind="reconstruct", bytes=rec, flops=0, launches=nf * L))
         stages.append(dict(name=f"frob_G{G}", kind="frob", bytes=fro, flops=0, launches=nf * L * 2))
         for m in m_values:

@@ -119,9 +119,31 @@ __device__ __forceinline__ double warp_sum(double v) {
 __host__ __device__ constexpr int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Programmatic dependent launch (device side): wait for the previous grid's
-// results before touching global memory, then let the next grid launch.
-__device__ __forceinline__ void pdl_enter() {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+// results before touching global memory, then let the next grid launch. The
+// order matters: a grid that has let its dependent launch has already seen
+// every earlier grid complete, which is what a dependent that starts early
+// (a forward after its own T = X.V kernel) relies on.
+//
+// The wait is an opaque asm statement to the compiler, and a load through a
+// `const __restrict__` kernel parameter counts as reading memory that nothing
+// else writes while the kernel runs, so the compiler may legally schedule such
+// a load before the wait -- and then read what the previous grid has not yet
+// written. after_wait() hides a pointer's origin behind an asm statement
+// ordered after the wait: every load through the returned value depends on it
+// and cannot move above the wait. pdl_enter(p, q, ...) does this for the
+// pointers it is given; every pointer whose target an earlier grid may write
+// must pass through one of the two.
+template <typename P>
+__device__ __forceinline__ void after_wait(P& p) {
+  asm volatile("" : "+l"(p) : : "memory");
+}
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+template <typename... P>
+__device__ __forceinline__ void pdl_enter(P&... ptrs) {
+  pdl_wait();
+  (after_wait(ptrs), ...);
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 

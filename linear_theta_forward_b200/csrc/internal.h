@@ -46,6 +46,12 @@ cudaError_t launch_reconstruct_simt(const LaunchCtx& c, theta_dtype dt, const fl
                                     const void* W0, const void* U, const void* V, int64_t O,
                                     int64_t I, int r, void* W_out);
 
+// ---- few-token forward on CUDA cores (gemv_kernels.cu): bf16
+int forward_gemv_max_tokens();
+cudaError_t launch_forward_gemv(const LaunchCtx& c, const void* X, const void* W0, const float* s, const void* U,
+                                const void* t_hi, const void* t_lo, int64_t M, int64_t O, int64_t I, int r, void* Y,
+                                bool early);
+
 // ---- tensor-core paths (umma_kernels.cu): bf16
 size_t forward_umma_workspace_bytes(int64_t M, int r);
 // Returns THETA_OK or a theta_status; CUDA errors are reported via *cuda_err.

@@ -85,7 +85,7 @@ template <typename T, int TPR, int VPT>
 __global__ void __launch_bounds__(kThreads)
 rowscale_band_kernel(const T* __restrict__ W0, PtrTable w, MutPtrTable s_out, MutPtrTable r_out,
                      int n, int64_t O, int64_t I, int write_r) {
-  pdl_enter();
+  pdl_enter(W0);
   using V = Vec<T>;
   using R = typename V::raw;
   constexpr int GROUPS = kThreads / TPR;
@@ -171,7 +171,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 rowscale_band_scalar_kernel(const T* __restrict__ W0, PtrTable w, MutPtrTable s_out,
                             MutPtrTable r_out, int n, int64_t O, int64_t I, int write_r) {
-  pdl_enter();
+  pdl_enter(W0);
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (kThreads / 32);
   for (int64_t o = (int64_t)blockIdx.x * (kThreads / 32) + threadIdx.x / 32; o < O; o += warps) {
@@ -201,7 +201,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 residual_vec_kernel(const T* __restrict__ w, const T* __restrict__ W0, const float* __restrict__ s,
                     int64_t nv_row, int64_t nvec, T* __restrict__ R) {
-  pdl_enter();
+  pdl_enter(w, W0, s);
   using V = Vec<T>;
   using Rw = typename V::raw;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -220,7 +220,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 residual_scalar_kernel(const T* __restrict__ w, const T* __restrict__ W0, const float* __restrict__ s,
                        int64_t I, int64_t count, T* __restrict__ R) {
-  pdl_enter();
+  pdl_enter(w, W0, s);
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += stride)
     R[i] = from_f32<T>(fmaf(-s[i / I], to_f32(W0[i]), to_f32(w[i])));
@@ -233,7 +233,7 @@ template <typename T>
 __global__ void __launch_bounds__(kThreads)
 frob_partial_kernel(const T* __restrict__ A, const T* __restrict__ B, int64_t nvec, int64_t count,
                     double* __restrict__ ws) {
-  pdl_enter();
+  pdl_enter(A, B);
   using V = Vec<T>;
   using R = typename V::raw;
   double num = 0.0, den = 0.0;
@@ -279,7 +279,7 @@ frob_partial_kernel(const T* __restrict__ A, const T* __restrict__ B, int64_t nv
 
 __global__ void __launch_bounds__(kThreads) frob_final_kernel(const double* __restrict__ ws, int nb,
                                                               double* __restrict__ out) {
-  pdl_enter();
+  pdl_enter(ws);
   double num = 0.0, den = 0.0;
   for (int k = threadIdx.x; k < nb; k += blockDim.x) {
     num += ws[2 * k];

@@ -123,14 +123,15 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // Programmatic dependent launch. Normally every thread waits here for the
-  // previous grid before touching global memory. A forward launched right
-  // after its own T = X.V kernel starts early instead: that kernel waited for
-  // all earlier work before it let this grid launch, and it writes only T, so
-  // W0, X and s may be streamed at once; only the loads of T (the producer's
-  // rank phase) and the epilogue wait.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // previous grid before touching global memory, and only then lets the next
+  // grid launch -- so a grid that lets its dependent start has itself seen
+  // all earlier work complete. A forward launched right after its own
+  // T = X.V kernel relies on exactly that: it starts early, streaming W0, X
+  // and s at once (that kernel writes only T), and waits only before the
+  // loads of T (the producer's rank phase) and in the epilogue.
   const bool early = MODE == MODE_FORWARD && args.early_start;
   if (!early) asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   auto give_up = [&]() {
     record_timeout(args.err);
@@ -319,7 +320,7 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
 // s (.) W0 for rank 0 (no tensor-core work).
 __global__ void __launch_bounds__(256) scale_rows_kernel(const float* __restrict__ s, const bf16* __restrict__ W0,
                                                          int64_t I, int64_t nvec, bf16* __restrict__ out) {
-  pdl_enter();
+  pdl_enter(s, W0);
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   const int64_t per_row = I / 8;
   for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < nvec; v += stride) {
@@ -382,7 +383,7 @@ recon_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  pdl_enter();
+  pdl_enter(s);
 
   if (threadIdx.x == 0) {
     ptx::mbar_arrive_expect_tx(bar_uv, 2 * C::kOpBytes);
@@ -530,10 +531,24 @@ cudaError_t prepare_kernel(KernelInfo* info, Kern kern, int threads, int smem, i
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
-  int blocks = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, threads, smem);
+  // Co-resident CTAs per SM, from shared memory (the binding limit for these
+  // kernels; the occupancy API under-reports kernels that use cluster
+  // instructions). Tensor memory must cover all of them, or allocation
+  // would stall.
+  int dev_smem = 0, reserved = 0;
+  e = cudaDeviceGetAttribute(&dev_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, 0);
   if (e != cudaSuccess) return e;
-  if (blocks < 1 || blocks * tmem_cols > 512) return cudaErrorInvalidConfiguration;
+  e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, 0);
+  if (e != cudaSuccess) return e;
+  int blocks = dev_smem / (smem + reserved);
+  const int by_threads = 2048 / threads;
+  if (blocks > by_threads) blocks = by_threads;
+  if (blocks < 1) return cudaErrorInvalidConfiguration;
+  if (blocks * tmem_cols > 512) blocks = 512 / tmem_cols;  // never counted on beyond tensor memory
+  int api_blocks = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&api_blocks, kern, threads, smem);
+  if (e != cudaSuccess) return e;
+  if (api_blocks * tmem_cols > 512) return cudaErrorInvalidConfiguration;
   info->blocks_per_sm = blocks;
   info->max_cluster = 1;
   if (clusters) {
@@ -640,6 +655,15 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
       *ce = e;
       return THETA_ERR_CUDA;
     }
+  }
+  // ---- a handful of tokens: a sequential sweep over W0 on CUDA cores
+  if (M <= forward_gemv_max_tokens()) {
+    e = launch_forward_gemv(c, X, W0, s, U, t_hi, t_lo, M, O, I, r, Y, r > 0);
+    if (e != cudaSuccess) {
+      *ce = e;
+      return THETA_ERR_CUDA;
+    }
+    return THETA_OK;
   }
   // ---- Y = s * (X . W0^T) + T . U^T, swap-AB: W0 rows are the MMA M side
   const int BN = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 256 ? 128 : 256;
