@@ -131,7 +131,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except (OSError, FileNotFoundError):
@@ -201,8 +201,12 @@ def result_line(*, value, unit, n_gpus, steps, warmup, ms_per_step, extra):
 class Workload:
     """All device tensors of one step, and the stage call lists."""
 
-    def __init__(self, theta, torch, seed=0, model=MODEL, r=RANK):
+    def __init__(self, theta, torch, seed=0, model=MODEL, r=RANK, streams=1):
         self.theta, self.torch = theta, torch
+        # independent calls of a stage (layers, families) spread round-robin
+        # over this many streams; each stream has its own workspaces
+        self.nstreams = streams
+        self.side = [torch.cuda.Stream() for _ in range(streams)] if streams > 1 else []
         self.model, self.r, self.L = model, r, model.num_layers
         dev = "cuda"
         bf = torch.bfloat16
@@ -222,42 +226,60 @@ class Workload:
                   for m in M_VALUES for fam, (O, _) in model.shapes.items() for l in range(L)}
         self.frob_out = torch.zeros(len(G_VALUES), len(model.shapes), L, dtype=torch.float64, device=dev)
         fb = theta.theta_workspace_size(theta.THETA_OP_FROB_ERROR, 1, 1, 1, 0, theta.THETA_BF16)
-        self.frob_ws = torch.empty(fb, dtype=torch.uint8, device=dev)
+        self.frob_ws = [torch.empty(fb, dtype=torch.uint8, device=dev) for _ in range(streams)]
         wb = max(theta.theta_workspace_size(theta.THETA_OP_LINEAR_FORWARD, m, O, I, r, theta.THETA_BF16)
                  for m in M_VALUES for (O, I) in model.shapes.values())
-        self.fwd_ws = torch.empty(max(wb, 256), dtype=torch.uint8, device=dev)
+        self.fwd_ws = [torch.empty(max(wb, 256), dtype=torch.uint8, device=dev) for _ in range(streams)]
         self.bands = {G: theta.theta_band_index(L, G)[0] for G in G_VALUES}
 
     # stage bodies ------------------------------------------------------
+    def _fan_out(self, calls):
+        """Runs calls(k) with k the stream slot: all on the current stream,
+        or forked round-robin over the side streams and joined back."""
+        if not self.side:
+            for c in calls:
+                c(0)
+            return
+        torch = self.torch
+        main = torch.cuda.current_stream()
+        for st in self.side:
+            st.wait_stream(main)
+        for i, c in enumerate(calls):
+            k = i % len(self.side)
+            with torch.cuda.stream(self.side[k]):
+                c(k)
+        for st in self.side:
+            main.wait_stream(st)
+
     def prelude(self, G):
         t = self.theta
-        for fam in self.model.shapes:
-            t.theta_decompose_prelude(self.W[fam], G, self.W0[fam][:G], self.s[fam], self.R[fam])
+        self._fan_out([lambda k, fam=fam: t.theta_decompose_prelude(self.W[fam], G, self.W0[fam][:G], self.s[fam],
+                                                                     self.R[fam])
+                       for fam in self.model.shapes])
 
     def reconstruct(self, G):
         t = self.theta
-        for fam in self.model.shapes:
-            band = self.bands[G]
-            for l in range(self.L):
-                t.theta_reconstruct(self.s[fam][l], self.W0[fam][band[l]], self.U[fam][l], self.V[fam][l],
-                                    self.rec[fam][l])
+        band = self.bands[G]
+        self._fan_out([lambda k, fam=fam, l=l: t.theta_reconstruct(self.s[fam][l], self.W0[fam][band[l]],
+                                                                    self.U[fam][l], self.V[fam][l],
+                                                                    self.rec[fam][l])
+                       for fam in self.model.shapes for l in range(self.L)])
 
     def frob(self, G):
         t = self.theta
         gi = G_VALUES.index(G)
-        for fi, fam in enumerate(self.model.shapes):
-            for l in range(self.L):
-                t.theta_frob_error(self.W[fam][l], self.rec[fam][l], self.frob_out[gi, fi, l:l + 1],
-                                   self.frob_ws)
+        self._fan_out([lambda k, fi=fi, fam=fam, l=l: t.theta_frob_error(self.W[fam][l], self.rec[fam][l],
+                                                                          self.frob_out[gi, fi, l:l + 1],
+                                                                          self.frob_ws[k])
+                       for fi, fam in enumerate(self.model.shapes) for l in range(self.L)])
 
     def forward(self, G, m):
         t = self.theta
         band = self.bands[G]
-        for fam, (O, I) in self.model.shapes.items():
-            X = self.X[(m, I)]
-            for l in range(self.L):
-                t.theta_linear_forward(X, self.W0[fam][band[l]], self.s[fam][l], self.U[fam][l], self.V[fam][l],
-                                       self.Y[(m, fam, l)], self.fwd_ws)
+        self._fan_out([lambda k, fam=fam, I=I, l=l: t.theta_linear_forward(
+            self.X[(m, I)], self.W0[fam][band[l]], self.s[fam][l], self.U[fam][l], self.V[fam][l],
+            self.Y[(m, fam, l)], self.fwd_ws[k])
+            for fam, (O, I) in self.model.shapes.items() for l in range(self.L)])
 
     def stage_fns(self):
         fns = []
@@ -406,7 +428,7 @@ def run_gpu(args):
     import linear_theta_forward_b200 as theta
 
     peaks = measured_peaks()
-    wl = Workload(theta, torch, seed=rank)
+    wl = Workload(theta, torch, seed=rank, streams=args.streams)
     stages = step_accounting()
     fns = wl.stage_fns()
     assert len(fns) == len(stages)
@@ -505,7 +527,7 @@ def run_gpu(args):
                                           "G": list(G_VALUES), "rank": RANK, "M": list(M_VALUES),
                                           "global_batch": max(M_VALUES), "seq_len": 1,
                                           "parallelism": f"independent replicas x{world}",
-                                          "graphs": not args.no_graph,
+                                          "graphs": not args.no_graph, "streams": args.streams,
                                           "l2": "inputs larger than L2 (>10 GB touched per step); no flush"},
                                "parts": parts,
                                "roofline": roofline,
@@ -564,15 +586,25 @@ def run_op(args):
     seed = 0
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     if args.op == "forward":
+        # --b2b: calls cycle over --bufs independent problems (like the layers
+        # of a model), so no call finds its W0 in L2
+        nbuf = args.bufs if args.b2b else 1
         X = syn.device_normal((M, I), 1.0, seed, "X", M, I)
-        W0 = syn.device_normal((O, I), 0.02, seed, "W0", O, I)
-        s = 1.0 + syn.device_normal((O,), 0.05, seed, "s", O, dtype="f32")
-        U = syn.device_normal((O, r), 0.01, seed, "U", O, r) if r else None
-        V = syn.device_normal((I, r), 0.01, seed, "V", I, r) if r else None
-        Y = torch.empty(M, O, dtype=torch.bfloat16, device="cuda")
+        probs = []
+        for k in range(nbuf):
+            W0 = syn.device_normal((O, I), 0.02, seed + k, "W0", O, I)
+            s = 1.0 + syn.device_normal((O,), 0.05, seed + k, "s", O, dtype="f32")
+            U = syn.device_normal((O, r), 0.01, seed + k, "U", O, r) if r else None
+            V = syn.device_normal((I, r), 0.01, seed + k, "V", I, r) if r else None
+            probs.append((W0, s, U, V, torch.empty(M, O, dtype=torch.bfloat16, device="cuda")))
         nb = theta.theta_workspace_size(theta.THETA_OP_LINEAR_FORWARD, M, O, I, r, theta.THETA_BF16)
         ws = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
-        call = lambda: theta.theta_linear_forward(X, W0, s, U, V, Y, ws)  # noqa: E731
+        turn = [0]
+
+        def call():
+            W0, s, U, V, Y = probs[turn[0] % nbuf]
+            turn[0] += 1
+            theta.theta_linear_forward(X, W0, s, U, V, Y, ws)
         nbytes, nflops = bytes_forward(M, O, I, r), flops_forward(M, O, I, r)
     elif args.op == "reconstruct":
         W0 = syn.device_normal((O, I), 0.02, seed, "W0", O, I)
@@ -603,20 +635,36 @@ def run_op(args):
         call()
     torch.cuda.synchronize()
     theta.theta_device_status()
-    times = []
-    for _ in range(args.iters):
-        flush.fill_(1)
+    if args.b2b:
+        # calls back to back between one pair of events; only meaningful
+        # for HBM when one call moves well over the 126 MB L2
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record()
-        call()
+        for _ in range(args.iters):
+            call()
         b.record()
         torch.cuda.synchronize()
-        times.append(a.elapsed_time(b))
+        ms = a.elapsed_time(b) / args.iters
+        l2 = "calls back to back, no flush (mean of %d)" % args.iters
+        if args.op == "forward":
+            l2 += ", cycling over %d independent problems" % args.bufs
+    else:
+        times = []
+        for _ in range(args.iters):
+            flush.fill_(1)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            call()
+            b.record()
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = statistics.median(times)
+        l2 = "flushed (256 MiB write) before every call"
     theta.theta_device_status()
-    ms = statistics.median(times)
     line = {"op": args.op, "shape": {"M": M, "O": O, "I": I, "rank": r, "layers": L, "G": G}, "dtype": "bf16",
-            "ms": round(ms, 5), "iters": args.iters, "l2": "flushed (256 MiB write) before every call",
+            "ms": round(ms, 5), "iters": args.iters, "l2": l2,
             "GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1),
             "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4), "algorithmic_bytes": nbytes}
     if nflops:
@@ -629,10 +677,11 @@ def run_op(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
+    ap.add_argument("--streams", type=int, default=16, help="streams the independent calls of a stage spread over")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -647,6 +696,8 @@ def main(argv=None):
     ap.add_argument("--layers", type=int, default=4)
     ap.add_argument("--G", type=int, default=1)
     ap.add_argument("--iters", type=int, default=20)
+    ap.add_argument("--b2b", action="store_true", help="--op: time --iters calls back to back (no L2 flush)")
+    ap.add_argument("--bufs", type=int, default=4, help="--op forward --b2b: independent problems cycled over")
     ap.add_argument("--no-residual", action="store_true", help="--op prelude: skip the residual output")
     args = ap.parse_args(argv)
     if args.op:

@@ -46,11 +46,15 @@ cudaError_t launch_reconstruct_simt(const LaunchCtx& c, theta_dtype dt, const fl
                                     const void* W0, const void* U, const void* V, int64_t O,
                                     int64_t I, int r, void* W_out);
 
-// ---- few-token forward on CUDA cores (gemv_kernels.cu): bf16
+// ---- few-token forward on CUDA cores (gemv_kernels.cu): bf16. Returns false
+// without launching when the problem does not fit (the caller takes the tile
+// path); launch errors come back in *e.
+// It launches its own T = X.V kernel; ws holds that kernel's partial sums.
 int forward_gemv_max_tokens();
-cudaError_t launch_forward_gemv(const LaunchCtx& c, const void* X, const void* W0, const float* s, const void* U,
-                                const void* t_hi, const void* t_lo, int64_t M, int64_t O, int64_t I, int r, void* Y,
-                                bool early);
+size_t forward_gemv_workspace_bytes(int64_t M, int r);
+bool launch_forward_gemv(const LaunchCtx& c, const void* X, const void* W0, const float* s, const void* U,
+                         const void* V, int64_t M, int64_t O, int64_t I, int r, void* Y, void* ws,
+                         cudaError_t* e);
 
 // ---- tensor-core paths (umma_kernels.cu): bf16
 size_t forward_umma_workspace_bytes(int64_t M, int r);

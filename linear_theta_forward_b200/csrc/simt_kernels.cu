@@ -33,13 +33,29 @@ __device__ __forceinline__ void load_tile(float (*dst)[BM + 1], const T* __restr
   }
 }
 
+// Sums of kChain consecutive products are formed on their own and then added
+// to the running total, so no fp32 rounding chain grows beyond about
+// kChain + K / kChain additions (a plain running sum over K = 16K drifts past
+// the 1e-5 relative tolerance of the fp32 path).
+constexpr int kChain = 256;
+
 template <typename TA, typename TB>
 __device__ __forceinline__ void accumulate(float (&acc)[4][4], const TA* __restrict__ A,
                                            const TB* __restrict__ B, int64_t Ma, int64_t Nb,
                                            int64_t K, int64_t a0, int64_t b0,
                                            float (*As)[BM + 1], float (*Bs)[BM + 1]) {
   const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;
+  float part[4][4] = {};
   for (int64_t k0 = 0; k0 < K; k0 += BK) {
+    if (k0 % kChain == 0 && k0 > 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[i][j] += part[i][j];
+          part[i][j] = 0.f;
+        }
+    }
     load_tile(As, A, Ma, K, a0, k0);
     load_tile(Bs, B, Nb, K, b0, k0);
     __syncthreads();
@@ -54,10 +70,14 @@ __device__ __forceinline__ void accumulate(float (&acc)[4][4], const TA* __restr
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(av[i], bv[j], part[i][j]);
     }
     __syncthreads();
   }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
 }
 
 // Y[M, O] = s (.) (X . W0^T) + T . U^T with T = X . V precomputed in fp32.
@@ -122,7 +142,12 @@ xv_simt_kernel(const T* __restrict__ X, const T* __restrict__ V, int64_t M, int6
     float acc = 0.f;
     if (j < r) {
       const T* x = X + m * I;
-      for (int64_t i = g; i < I; i += 8) acc = fmaf(to_f32(x[i]), to_f32(V[i * r + j]), acc);
+      for (int64_t i0 = 0; i0 < I; i0 += 8 * kChain) {  // chains of kChain products
+        float part = 0.f;
+        const int64_t i1 = i0 + 8 * kChain < I ? i0 + 8 * kChain : I;
+        for (int64_t i = i0 + g; i < i1; i += 8) part = fmaf(to_f32(x[i]), to_f32(V[i * r + j]), part);
+        acc += part;
+      }
     }
     part[g][lane] = acc;
     __syncthreads();

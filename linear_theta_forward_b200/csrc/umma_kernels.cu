@@ -592,7 +592,12 @@ cudaError_t launch_tile_kernel(const LaunchCtx& c, const CUtensorMap& a1, const 
   cudaError_t e = prepare_kernel(&info[c.device], kern, kThreads, C::kSmemBytes, C::kTmemCols, true);
   if (e != cudaSuccess) return e;
   const int64_t tiles = (int64_t)m_tiles * n_tiles;
-  args.splits = pick_splits(tiles, args.kb1, c.num_sms * info[c.device].blocks_per_sm, info[c.device].max_cluster);
+  // Tiles of 64 or more columns keep the tensor pipe busy: a second CTA on
+  // the same SM adds no throughput, only split-K reduction work, so they
+  // count one CTA per SM. Narrow (decode) tiles are bound by memory latency
+  // and count every co-resident CTA.
+  const int capacity = c.num_sms * (BN >= 64 ? 1 : info[c.device].blocks_per_sm);
+  args.splits = pick_splits(tiles, args.kb1, capacity, info[c.device].max_cluster);
   return launch_pdl(kern, dim3((unsigned)(n_tiles * args.splits), (unsigned)m_tiles, 1), dim3(kThreads), C::kSmemBytes,
                     c.stream, args.splits, a1, b1, a2, b2, b3, args);
 }
@@ -613,7 +618,8 @@ cudaError_t launch_recon(const LaunchCtx& c, const CUtensorMap& mU, const CUtens
 
 size_t forward_umma_workspace_bytes(int64_t M, int r) {
   const size_t half = ((size_t)M * r * 2 + 255) / 256 * 256;
-  return 2 * half;
+  const size_t gemv = forward_gemv_workspace_bytes(M, r);
+  return 2 * half > gemv ? 2 * half : gemv;
 }
 
 int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const float* s, const void* U,
@@ -622,12 +628,20 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
   *ce = cudaSuccess;
   if (O > (int64_t)65535 * kBM || M > ((int64_t)1 << 30) || I > ((int64_t)1 << 31) - 64 || r > 256)
     return THETA_ERR_UNSUPPORTED;
+  cudaError_t e = cudaSuccess;
+  // ---- a handful of tokens: a sequential sweep over W0 on CUDA cores
+  if (M <= forward_gemv_max_tokens() && launch_forward_gemv(c, X, W0, s, U, V, M, O, I, r, Y, ws, &e)) {
+    if (e != cudaSuccess) {
+      *ce = e;
+      return THETA_ERR_CUDA;
+    }
+    return THETA_OK;
+  }
   const int kb = (int)ceil_div(I, kBK);
   bf16* t_hi = nullptr;
   bf16* t_lo = nullptr;
   CUtensorMap mX, mW0, mU, mThi, mTlo, mV;
   int st;
-  cudaError_t e = cudaSuccess;
   if (r > 0) {
     t_hi = static_cast<bf16*>(ws);
     t_lo = reinterpret_cast<bf16*>(static_cast<uint8_t*>(ws) + forward_umma_workspace_bytes(M, r) / 2);
@@ -655,15 +669,6 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
       *ce = e;
       return THETA_ERR_CUDA;
     }
-  }
-  // ---- a handful of tokens: a sequential sweep over W0 on CUDA cores
-  if (M <= forward_gemv_max_tokens()) {
-    e = launch_forward_gemv(c, X, W0, s, U, t_hi, t_lo, M, O, I, r, Y, r > 0);
-    if (e != cudaSuccess) {
-      *ce = e;
-      return THETA_ERR_CUDA;
-    }
-    return THETA_OK;
   }
   // ---- Y = s * (X . W0^T) + T . U^T, swap-AB: W0 rows are the MMA M side
   const int BN = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 256 ? 128 : 256;

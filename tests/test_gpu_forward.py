@@ -66,6 +66,15 @@ FORWARD_CASES = [
     (8, 136, 200, 192),
     (130, 264, 392, 256),
     (3, 1024, 6912, 16),     # deep K: split across a cluster
+    # one or two tokens (the CUDA-core sweep): ragged row ranges per CTA,
+    # long rows, maximum rank; three and four tokens take the tile path
+    (2, 4104, 1152, 64),
+    (4, 1000, 200, 8),
+    (2, 1000, 8200, 24),
+    (4, 304, 16392, 0),
+    (1, 24, 64, 8),
+    (3, 2056, 200, 256),
+    (4, 136, 24, 16),
 ]
 
 
@@ -79,7 +88,8 @@ def test_forward(lib, torch, dt, M, O, I, r):
 
 
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
-@pytest.mark.parametrize("M,O,I,r", [(16, 392, 328, 32), (200, 256, 1152, 64), (1, 1024, 1152, 64)])
+@pytest.mark.parametrize("M,O,I,r", [(16, 392, 328, 32), (200, 256, 1152, 64), (1, 1024, 1152, 64),
+                                     (4, 1024, 1152, 64), (2, 520, 9000, 32)])
 def test_forward_large_rank_term(lib, torch, dt, M, O, I, r):
     """U, V ~ N(0, 0.1): the rank term is comparable to the main term."""
     X, W0, s, U, V = bundle(M, O, I, r, dt, seed=7, uv_std=0.1)
