@@ -428,6 +428,9 @@ def run_gpu(args):
     import linear_theta_forward_b200 as theta
 
     peaks = measured_peaks()
+    # many independent calls in flight at once: no split-K
+    policy = theta.THETA_POLICY_THROUGHPUT if args.streams > 1 else theta.THETA_POLICY_LATENCY
+    theta.theta_set_policy(policy)
     wl = Workload(theta, torch, seed=rank, streams=args.streams)
     stages = step_accounting()
     fns = wl.stage_fns()
@@ -528,6 +531,7 @@ def run_gpu(args):
                                           "global_batch": max(M_VALUES), "seq_len": 1,
                                           "parallelism": f"independent replicas x{world}",
                                           "graphs": not args.no_graph, "streams": args.streams,
+                                          "policy": "throughput" if policy else "latency",
                                           "l2": "inputs larger than L2 (>10 GB touched per step); no flush"},
                                "parts": parts,
                                "roofline": roofline,

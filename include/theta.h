@@ -64,6 +64,12 @@ typedef enum {
   THETA_OP_LINEAR_FORWARD = 1
 } theta_op;
 
+/* How the tensor-core kernels size their grids (see theta_set_policy). */
+typedef enum {
+  THETA_POLICY_LATENCY = 0,   /* default: split K across a cluster so one call fills the GPU */
+  THETA_POLICY_THROUGHPUT = 1 /* one CTA per output tile: many calls run concurrently */
+} theta_policy;
+
 /* Library version (THETA_VERSION of the build). */
 int theta_version(void);
 
@@ -225,6 +231,26 @@ int theta_linear_forward_noalloc(const void* X, int64_t M, int64_t I, const void
  */
 int theta_workspace_size(int op, int64_t M, int64_t O, int64_t I, int rank, theta_dtype dt,
                          size_t* bytes);
+
+/*
+ * theta_set_policy -- grid sizing of the tensor-core kernels of
+ * theta_linear_forward (the T = X.V kernel and the main projection) for the
+ * calls that follow, process-wide. Not an operation of the method: a launch
+ * choice that does not change any result beyond floating-point summation
+ * order.
+ *   THETA_POLICY_LATENCY (default): when the output tiles of one call leave
+ *     SMs idle, K is split over a thread-block cluster and the partial tiles
+ *     are summed through distributed shared memory -- the fastest single call.
+ *   THETA_POLICY_THROUGHPUT: no split; every CTA owns a whole output tile.
+ *     For callers that keep the GPU busy with many independent calls on
+ *     several streams, where split-K's extra CTAs, cluster scheduling and
+ *     reductions cost more than they gain.
+ * Returns THETA_ERR_INVALID_ARG for any other value. Safe to call from any
+ * thread; calls already enqueued keep the policy they were launched with.
+ * theta_get_policy returns the current policy.
+ */
+int theta_set_policy(int policy);
+int theta_get_policy(void);
 
 /*
  * theta_device_status -- synchronises `stream`, then reads and clears the

@@ -19,13 +19,15 @@ __all__ = [
     "theta_version", "theta_status_string", "theta_last_error", "theta_band_index",
     "theta_band_mean", "theta_row_scale", "theta_residual", "theta_decompose_prelude",
     "theta_reconstruct", "theta_frob_error", "theta_linear_forward", "theta_workspace_size",
-    "theta_device_status", "theta_linear_forward_noalloc",
+    "theta_device_status", "theta_linear_forward_noalloc", "theta_set_policy", "theta_get_policy",
+    "THETA_POLICY_LATENCY", "THETA_POLICY_THROUGHPUT",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtheta.so")
 
 THETA_F32, THETA_BF16 = 0, 1
 THETA_OP_FROB_ERROR, THETA_OP_LINEAR_FORWARD = 0, 1
+THETA_POLICY_LATENCY, THETA_POLICY_THROUGHPUT = 0, 1
 THETA_MAX_LAYERS = 256
 
 _i32p = ctypes.POINTER(ctypes.c_int32)
@@ -36,6 +38,8 @@ _sz = ctypes.c_size_t
 
 _SIGNATURES = {
     "theta_version": (_int,),
+    "theta_set_policy": (_int, _int),
+    "theta_get_policy": (_int,),
     "theta_status_string": (ctypes.c_char_p, _int),
     "theta_last_error": (ctypes.c_char_p,),
     "theta_band_index": (_int, _int, _int, _i32p, _i32p),
@@ -240,6 +244,17 @@ def theta_linear_forward_noalloc(X, W0, s, U, V, Y, stream=None) -> None:
                                             _ptr(U, "U", optional=True), _ptr(V, "V", optional=True), rank,
                                             _dtype_code(X), _ptr(Y, "Y"), _stream(stream)),
            "theta_linear_forward_noalloc")
+
+
+def theta_set_policy(policy: int) -> None:
+    """Grid sizing of the tensor-core forward kernels for the calls that
+    follow: THETA_POLICY_LATENCY (split-K, default) or THETA_POLICY_THROUGHPUT
+    (one CTA per output tile, for many concurrent calls)."""
+    _check(_load().theta_set_policy(int(policy)), "theta_set_policy")
+
+
+def theta_get_policy() -> int:
+    return _load().theta_get_policy()
 
 
 def theta_device_status(stream=None) -> None:

@@ -14,6 +14,7 @@ struct LaunchCtx {
   unsigned* err;  // device error words of the current device
   int num_sms;
   int device;
+  int policy;  // theta_policy at the time of the call
 };
 
 // ---- streaming kernels (stream_kernels.cu)

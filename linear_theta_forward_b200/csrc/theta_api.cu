@@ -7,6 +7,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <string>
 
@@ -46,6 +47,8 @@ struct DeviceState {
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
 
+std::atomic<int> g_policy{THETA_POLICY_LATENCY};
+
 int make_ctx(void* stream, LaunchCtx* ctx) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -66,6 +69,7 @@ int make_ctx(void* stream, LaunchCtx* ctx) {
   }
   ctx->device = dev;
   ctx->stream = static_cast<cudaStream_t>(stream);
+  ctx->policy = g_policy.load(std::memory_order_relaxed);
   return THETA_OK;
 }
 
@@ -315,6 +319,15 @@ THETA_API int theta_workspace_size(int op, int64_t M, int64_t O, int64_t I, int 
   }
   return fail(THETA_ERR_INVALID_ARG, "theta_workspace_size: unknown op %d", op);
 }
+
+THETA_API int theta_set_policy(int policy) {
+  if (policy != THETA_POLICY_LATENCY && policy != THETA_POLICY_THROUGHPUT)
+    return fail(THETA_ERR_INVALID_ARG, "theta_set_policy: unknown policy %d", policy);
+  g_policy.store(policy, std::memory_order_relaxed);
+  return THETA_OK;
+}
+
+THETA_API int theta_get_policy(void) { return g_policy.load(std::memory_order_relaxed); }
 
 THETA_API int theta_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));

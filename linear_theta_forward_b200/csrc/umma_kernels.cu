@@ -597,7 +597,9 @@ cudaError_t launch_tile_kernel(const LaunchCtx& c, const CUtensorMap& a1, const 
   // count one CTA per SM. Narrow (decode) tiles are bound by memory latency
   // and count every co-resident CTA.
   const int capacity = c.num_sms * (BN >= 64 ? 1 : info[c.device].blocks_per_sm);
-  args.splits = pick_splits(tiles, args.kb1, capacity, info[c.device].max_cluster);
+  args.splits = c.policy == THETA_POLICY_THROUGHPUT
+                    ? 1
+                    : pick_splits(tiles, args.kb1, capacity, info[c.device].max_cluster);
   return launch_pdl(kern, dim3((unsigned)(n_tiles * args.splits), (unsigned)m_tiles, 1), dim3(kThreads), C::kSmemBytes,
                     c.stream, args.splits, a1, b1, a2, b2, b3, args);
 }

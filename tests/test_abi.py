@@ -97,3 +97,16 @@ def test_workspace_sizes(lib):
         assert b >= 300 * 24 * 4 and b % 256 == 0
     with pytest.raises(lib.ThetaError):
         lib.theta_workspace_size(99, 1, 1, 1, 0, lib.THETA_F32)
+
+
+def test_launch_policy_round_trip(lib):
+    assert lib.theta_get_policy() == lib.THETA_POLICY_LATENCY
+    try:
+        lib.theta_set_policy(lib.THETA_POLICY_THROUGHPUT)
+        assert lib.theta_get_policy() == lib.THETA_POLICY_THROUGHPUT
+        with pytest.raises(lib.ThetaError):
+            lib.theta_set_policy(7)
+        assert lib.theta_get_policy() == lib.THETA_POLICY_THROUGHPUT  # a rejected value changes nothing
+    finally:
+        lib.theta_set_policy(lib.THETA_POLICY_LATENCY)
+    assert lib.theta_get_policy() == lib.THETA_POLICY_LATENCY

@@ -100,6 +100,20 @@ def test_forward_large_rank_term(lib, torch, dt, M, O, I, r):
     assert_close(got, ref, dt, "Y")
 
 
+@pytest.mark.parametrize("M,O,I,r", [(3, 1024, 6912, 16), (16, 392, 328, 32), (64, 1024, 1152, 32),
+                                     (600, 256, 1152, 32), (40, 256, 264, 128)])
+def test_forward_throughput_policy(lib, torch, M, O, I, r):
+    """Without split-K (every CTA owns a whole tile) the result is the same."""
+    X, W0, s, U, V = bundle(M, O, I, r, "bf16", seed=5)
+    ref = oracle.linear_forward(X, W0, s, U, V)
+    lib.theta_set_policy(lib.THETA_POLICY_THROUGHPUT)
+    try:
+        got = run_forward(lib, torch, X, W0, s, U, V, "bf16")
+    finally:
+        lib.theta_set_policy(lib.THETA_POLICY_LATENCY)
+    assert_close(got, ref, "bf16", "Y")
+
+
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
 def test_forward_rank0_is_scaled_shared_block(lib, torch, dt):
     X, W0, s, U, V = bundle(9, 264, 520, 0, dt, seed=3)
