@@ -27,10 +27,13 @@ cudaError_t launch_rowscale_band(const LaunchCtx& c, theta_dtype dt, const void*
 cudaError_t launch_residual(const LaunchCtx& c, theta_dtype dt, const void* w, const void* W0,
                             const float* s, int64_t O, int64_t I, void* R);
 // ---- prelude pipeline (prelude_kernels.cu): every band of a family in one
-// launch. band_mode: bands of <= 4 layers, forms W0, s and R in one pass;
-// otherwise reads the already-formed W0 and writes s and R. Returns false
-// without launching when the problem does not fit the pipeline.
-bool launch_prelude_pipe(const LaunchCtx& c, theta_dtype dt, bool band_mode, const void* const* w, int L, int G,
+// launch. PRELUDE_BAND: bands of <= 4 layers, W0, s and R in one pass;
+// PRELUDE_TWO_PASS: longer bands, W0 from a first pass over the band's rows,
+// s and R from a second (L2-resident) pass; PRELUDE_ROW: reads the
+// already-formed W0 and writes s and R. Returns false without launching when
+// the problem does not fit the chosen kernel.
+enum { PRELUDE_ROW = 0, PRELUDE_BAND = 1, PRELUDE_TWO_PASS = 2 };
+bool launch_prelude_pipe(const LaunchCtx& c, theta_dtype dt, int mode, const void* const* w, int L, int G,
                          const int32_t* band_start, const int32_t* band_of_layer, void* const* W0,
                          float* const* s, void* const* R, int64_t O, int64_t I, cudaError_t* e);
 size_t frob_workspace_bytes();

@@ -165,7 +165,7 @@ THETA_API int theta_row_scale(const void* weight, const void* W0, int64_t O, int
   void* w0[1] = {const_cast<void*>(W0)};
   const int32_t band_start[2] = {0, 1}, band_of_layer[1] = {0};
   cudaError_t pe = cudaSuccess;
-  if (launch_prelude_pipe(c, dt, false, w, 1, 1, band_start, band_of_layer, w0, sp, nullptr, O, I, &pe)) {
+  if (launch_prelude_pipe(c, dt, PRELUDE_ROW, w, 1, 1, band_start, band_of_layer, w0, sp, nullptr, O, I, &pe)) {
     CHECK_LAUNCH(pe, "theta_row_scale launch");
     return THETA_OK;
   }
@@ -208,8 +208,14 @@ THETA_API int theta_decompose_prelude(const void* const* weights, int num_layers
   const int nmax = (num_layers + G - 1) / G;
   cudaError_t pe = cudaSuccess;
   // bands of <= 4 layers: one pass over the family forms W0, s and R
-  if (nmax <= 4 && launch_prelude_pipe(c, dt, true, weights, num_layers, G, band_start, band_of_layer, W0, s,
-                                       residual, O, I, &pe)) {
+  if (nmax <= 4 && launch_prelude_pipe(c, dt, PRELUDE_BAND, weights, num_layers, G, band_start, band_of_layer, W0,
+                                       s, residual, O, I, &pe)) {
+    CHECK_LAUNCH(pe, "prelude launch");
+    return THETA_OK;
+  }
+  // longer bands: two passes over each band's rows, the second from L2
+  if (nmax > 4 && launch_prelude_pipe(c, dt, PRELUDE_TWO_PASS, weights, num_layers, G, band_start, band_of_layer,
+                                      W0, s, residual, O, I, &pe)) {
     CHECK_LAUNCH(pe, "prelude launch");
     return THETA_OK;
   }
@@ -217,8 +223,8 @@ THETA_API int theta_decompose_prelude(const void* const* weights, int num_layers
     const int first = band_start[b], n = band_start[b + 1] - band_start[b];
     CHECK_LAUNCH(launch_band_mean(c, dt, weights + first, n, O, I, W0[b]), "band mean launch");
   }
-  if (launch_prelude_pipe(c, dt, false, weights, num_layers, G, band_start, band_of_layer, W0, s, residual, O, I,
-                          &pe)) {
+  if (launch_prelude_pipe(c, dt, PRELUDE_ROW, weights, num_layers, G, band_start, band_of_layer, W0, s, residual, O,
+                          I, &pe)) {
     CHECK_LAUNCH(pe, "row scale launch");
     return THETA_OK;
   }

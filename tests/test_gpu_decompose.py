@@ -99,7 +99,12 @@ def test_zero_w0_row_gives_zero_scale(lib, torch):
                                         ("bf16", 6, 1, 9, 5376),
                                         ("bf16", 8, 2, 33, 5376),     # one-pass prelude, 4-layer bands
                                         ("bf16", 2, 2, 20, 21504),    # one-pass prelude, widest rows
-                                        ("f32", 3, 1, 21, 1000)])
+                                        ("f32", 3, 1, 21, 1000),
+                                        # two-pass prelude (bands of more than 4 layers)
+                                        ("f32", 9, 2, 19, 1000),
+                                        ("bf16", 60, 1, 3, 5376),
+                                        ("bf16", 11, 2, 130, 1152),
+                                        ("bf16", 12, 1, 5, 21504)])  # rows too long: band mean + row pass
 def test_decompose_prelude(lib, torch, dt, L, G, O, I):
     w = weights(L, O, I, dt, seed=L * G)
     ws = [dev(w[i], dt) for i in range(L)]
