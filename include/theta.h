@@ -30,7 +30,9 @@
  *     (I, O and r multiples of 8); otherwise they return THETA_ERR_ALIGNMENT.
  *   - Kernels bound every wait they make. A wait that runs out records a flag
  *     on the device and the kernel returns early; theta_device_status() reports
- *     it as THETA_ERR_TIMEOUT.
+ *     it as THETA_ERR_TIMEOUT and clears it. While the flag is set, kernels
+ *     with waits skip their work (outputs undefined) so that a fault does not
+ *     cost every later CTA its own wait limit.
  *   - theta_last_error() gives a message for the last failing call on the
  *     calling thread.
  */
@@ -251,6 +253,17 @@ int theta_workspace_size(int op, int64_t M, int64_t O, int64_t I, int rank, thet
  */
 int theta_set_policy(int policy);
 int theta_get_policy(void);
+
+/*
+ * theta_selftest_wait_timeout -- exercises the failure path of the bounded
+ * device waits (not an operation of the method): enqueues one kernel whose
+ * wait on a barrier that nothing completes gives up after limit_ms
+ * milliseconds (1..2000) and records the timeout flag, exactly as a kernel
+ * whose producer stopped would. The next theta_device_status() on `stream`
+ * returns THETA_ERR_TIMEOUT and clears the flag; the CUDA context stays
+ * usable. Returns THETA_ERR_INVALID_ARG for a limit outside the range.
+ */
+int theta_selftest_wait_timeout(unsigned limit_ms, void* stream);
 
 /*
  * theta_device_status -- synchronises `stream`, then reads and clears the

@@ -20,7 +20,7 @@ __all__ = [
     "theta_band_mean", "theta_row_scale", "theta_residual", "theta_decompose_prelude",
     "theta_reconstruct", "theta_frob_error", "theta_linear_forward", "theta_workspace_size",
     "theta_device_status", "theta_linear_forward_noalloc", "theta_set_policy", "theta_get_policy",
-    "THETA_POLICY_LATENCY", "THETA_POLICY_THROUGHPUT",
+    "theta_selftest_wait_timeout", "THETA_POLICY_LATENCY", "THETA_POLICY_THROUGHPUT",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtheta.so")
@@ -39,6 +39,7 @@ _sz = ctypes.c_size_t
 _SIGNATURES = {
     "theta_version": (_int,),
     "theta_set_policy": (_int, _int),
+    "theta_selftest_wait_timeout": (_int, ctypes.c_uint, _vp),
     "theta_get_policy": (_int,),
     "theta_status_string": (ctypes.c_char_p, _int),
     "theta_last_error": (ctypes.c_char_p,),
@@ -255,6 +256,12 @@ def theta_set_policy(policy: int) -> None:
 
 def theta_get_policy() -> int:
     return _load().theta_get_policy()
+
+
+def theta_selftest_wait_timeout(limit_ms: int, stream=None) -> None:
+    """Enqueues one bounded wait that nothing completes; the next
+    theta_device_status() raises THETA_ERR_TIMEOUT."""
+    _check(_load().theta_selftest_wait_timeout(int(limit_ms), _stream(stream)), "theta_selftest_wait_timeout")
 
 
 def theta_device_status(stream=None) -> None:

@@ -35,6 +35,15 @@ __device__ __forceinline__ void record_timeout(unsigned* err) {
   if (err) atomicExch(err + ERR_WORD_TIMEOUT, 1u);
 }
 
+// 1 if some wait on this device ran out since theta_device_status() last
+// cleared the flag. Kernels with bounded waits start with their abort flag
+// set to this, so after one timeout the rest give up at once (their results
+// are undefined until the status is read) instead of each waiting out its
+// own limit.
+__device__ __forceinline__ int prior_timeout(const unsigned* err) {
+  return (err && *reinterpret_cast<const volatile unsigned*>(err + ERR_WORD_TIMEOUT)) ? 1 : 0;
+}
+
 // ------------------------------------------------------------- element I/O
 // 16-byte vectors: 8 bf16 or 4 fp32 elements.
 template <typename T>

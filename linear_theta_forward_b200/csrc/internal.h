@@ -66,6 +66,8 @@ size_t forward_umma_workspace_bytes(int64_t M, int r);
 int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const float* s,
                         const void* U, const void* V, int64_t M, int64_t O, int64_t I, int r,
                         void* Y, void* ws, cudaError_t* cuda_err);
+// One bounded wait that nothing completes (gives up after limit_ms).
+cudaError_t launch_wait_selftest(const LaunchCtx& c, unsigned limit_ms);
 int launch_reconstruct_umma(const LaunchCtx& c, const float* s, const void* W0, const void* U,
                             const void* V, int64_t O, int64_t I, int r, void* W_out,
                             cudaError_t* cuda_err);

@@ -89,7 +89,7 @@ prelude_pipe_kernel(const __grid_constant__ PreludeArgs a) {
       ptx::mbar_init(&full[i], 1);
       ptx::mbar_init(&empty[i], kConsumers / 32);
     }
-    abort_flag = 0;
+    abort_flag = prior_timeout(a.err);
     ptx::fence_mbarrier_init();
   }
   __syncthreads();
@@ -304,7 +304,7 @@ prelude_band2_kernel(const __grid_constant__ PreludeArgs a) {
       ptx::mbar_init(&full[i], 1);
       ptx::mbar_init(&empty[i], kConsumers / 32);
     }
-    abort_flag = 0;
+    abort_flag = prior_timeout(a.err);
     ptx::fence_mbarrier_init();
   }
   __syncthreads();

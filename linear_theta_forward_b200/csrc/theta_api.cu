@@ -326,6 +326,16 @@ THETA_API int theta_workspace_size(int op, int64_t M, int64_t O, int64_t I, int 
   return fail(THETA_ERR_INVALID_ARG, "theta_workspace_size: unknown op %d", op);
 }
 
+THETA_API int theta_selftest_wait_timeout(unsigned limit_ms, void* stream) {
+  if (limit_ms < 1 || limit_ms > 2000)
+    return fail(THETA_ERR_INVALID_ARG, "theta_selftest_wait_timeout: limit %u ms outside [1, 2000]", limit_ms);
+  LaunchCtx c;
+  int st = make_ctx(stream, &c);
+  if (st) return st;
+  CHECK_LAUNCH(launch_wait_selftest(c, limit_ms), "theta_selftest_wait_timeout launch");
+  return THETA_OK;
+}
+
 THETA_API int theta_set_policy(int policy) {
   if (policy != THETA_POLICY_LATENCY && policy != THETA_POLICY_THROUGHPUT)
     return fail(THETA_ERR_INVALID_ARG, "theta_set_policy: unknown policy %d", policy);

@@ -111,7 +111,7 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
     }
     ptx::mbar_init(accum, 1);
     ptx::mbar_init(drain, 1);
-    *abort_flag = 0;
+    *abort_flag = prior_timeout(args.err);
     ptx::fence_mbarrier_init();
   }
   if (warp == 1) {
@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(256) scale_rows_kernel(const float* __restrict
 }
 
 // ------------------------------------------------------------- reconstruct
-// One 128 x 128 tile of W = diag(s).W0 + U.V^T. 128 threads: thread 0 issues
+// One 128 x kRecN tile of W = diag(s).W0 + U.V^T. 128 threads: thread 0 issues
 // the TMA loads (U and V rank blocks on one barrier, the W0 tile on another)
 // and the final TMA store; thread 32 issues the K = rank MMAs; then all four
 // warps read their 32-lane quarter of U.V^T from tensor memory, combine it
@@ -344,9 +344,12 @@ constexpr int kRecN = 128;  // columns of W per tile
 
 template <int KB>
 struct RecCfg {
-  static constexpr int kOpBytes = KB * kABytes;         // U or V: KB blocks of 128 rows x 64
-  static constexpr int kWBytes = 2 * kABytes;           // W0 / output tile: two 64-column boxes
-  static constexpr int kSmemBytes = 2 * kOpBytes + kWBytes + 1024 + 128;
+  static constexpr int kUBlock = kBM * 128;              // U: 128 rows x 64 rank columns (bf16)
+  static constexpr int kVBlock = kRecN * 128;            // V: kRecN rows x 64 rank columns
+  static constexpr int kUBytes = KB * kUBlock;
+  static constexpr int kVBytes = KB * kVBlock;
+  static constexpr int kWBytes = (kRecN / kBK) * kABytes;  // W0 / output tile: kRecN / 64 column boxes
+  static constexpr int kSmemBytes = kUBytes + kVBytes + kWBytes + 1024 + 128;
 };
 
 template <int KB>
@@ -358,8 +361,8 @@ recon_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sU = smem;
-  uint8_t* sV = smem + C::kOpBytes;
-  uint8_t* sW = sV + C::kOpBytes;
+  uint8_t* sV = smem + C::kUBytes;
+  uint8_t* sW = sV + C::kVBytes;
   uint64_t* bar_uv = reinterpret_cast<uint64_t*>(sW + C::kWBytes);
   uint64_t* bar_w = bar_uv + 1;
   uint64_t* bar_acc = bar_w + 1;
@@ -372,7 +375,7 @@ recon_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
     ptx::mbar_init(bar_uv, 1);
     ptx::mbar_init(bar_w, 1);
     ptx::mbar_init(bar_acc, 1);
-    *abort_flag = 0;
+    *abort_flag = prior_timeout(err);
     ptx::fence_mbarrier_init();
   }
   if (warp == 1) {
@@ -386,15 +389,15 @@ recon_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
   pdl_enter(s);
 
   if (threadIdx.x == 0) {
-    ptx::mbar_arrive_expect_tx(bar_uv, 2 * C::kOpBytes);
+    ptx::mbar_arrive_expect_tx(bar_uv, C::kUBytes + C::kVBytes);
 #pragma unroll
     for (int kb = 0; kb < KB; ++kb) {
-      ptx::tma_load_2d(sU + kb * kABytes, &tmU, bar_uv, kb * kBK, o0);
-      ptx::tma_load_2d(sV + kb * kABytes, &tmV, bar_uv, kb * kBK, i0);
+      ptx::tma_load_2d(sU + kb * C::kUBlock, &tmU, bar_uv, kb * kBK, o0);
+      ptx::tma_load_2d(sV + kb * C::kVBlock, &tmV, bar_uv, kb * kBK, i0);
     }
     ptx::mbar_arrive_expect_tx(bar_w, C::kWBytes);
-    ptx::tma_load_2d(sW, &tmW0, bar_w, i0, o0);
-    ptx::tma_load_2d(sW + kABytes, &tmW0, bar_w, i0 + kBK, o0);
+#pragma unroll
+    for (int bx = 0; bx < kRecN / kBK; ++bx) ptx::tma_load_2d(sW + bx * kABytes, &tmW0, bar_w, i0 + bx * kBK, o0);
   }
   bool mma_issued = false;
   if (threadIdx.x == 32) {
@@ -406,8 +409,8 @@ recon_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
       for (int kb = 0; kb < KB; ++kb)
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk)
-          ptx::umma_bf16(tmem, ptx::sdesc_sw128(ua + kb * kABytes + kk * 32, 16, 1024),
-                         ptx::sdesc_sw128(va + kb * kABytes + kk * 32, 16, 1024), idesc, (kb | kk) ? 1u : 0u);
+          ptx::umma_bf16(tmem, ptx::sdesc_sw128(ua + kb * C::kUBlock + kk * 32, 16, 1024),
+                         ptx::sdesc_sw128(va + kb * C::kVBlock + kk * 32, 16, 1024), idesc, (kb | kk) ? 1u : 0u);
       ptx::umma_commit(bar_acc);
       mma_issued = true;
     } else {
@@ -450,8 +453,9 @@ recon_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
   __syncthreads();
   if (threadIdx.x == 0) {
     if (!*abort_flag) {
-      ptx::tma_store_2d(&tmOut, sW, i0, o0);
-      if (i0 + kBK < I) ptx::tma_store_2d(&tmOut, sW + kABytes, i0 + kBK, o0);
+#pragma unroll
+      for (int bx = 0; bx < kRecN / kBK; ++bx)
+        if (i0 + bx * kBK < I) ptx::tma_store_2d(&tmOut, sW + bx * kABytes, i0 + bx * kBK, o0);
       ptx::bulk_commit();
       ptx::bulk_wait_read();
     } else {
@@ -616,7 +620,26 @@ cudaError_t launch_recon(const LaunchCtx& c, const CUtensorMap& mU, const CUtens
                     C::kSmemBytes, c.stream, 1, mU, mV, mW0, mOut, s, O, I, c.err);
 }
 
+// The failure path of every bounded wait, on purpose: one thread waits on an
+// mbarrier that nothing will complete, gives up after limit_ns, records the
+// timeout flag and returns; the host reads it through theta_device_status.
+__global__ void wait_selftest_kernel(unsigned* err, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int never;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    never = 0;
+    ptx::fence_mbarrier_init();
+    if (!ptx::mbar_wait(&bar, 0, &never, limit_ns)) record_timeout(err);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_wait_selftest(const LaunchCtx& c, unsigned limit_ms) {
+  wait_selftest_kernel<<<1, 32, 0, c.stream>>>(c.err, (unsigned long long)limit_ms * 1000000ull);
+  return cudaGetLastError();
+}
 
 size_t forward_umma_workspace_bytes(int64_t M, int r) {
   const size_t half = ((size_t)M * r * 2 + 255) / 256 * 256;
