@@ -77,6 +77,26 @@ def flops_forward(M, O, I, r):
     return 2 * M * (O * I + r * (I + O))
 
 
+def prelude_launches(L, G, I, b=BF16, num_sms=148):
+    """Kernel launches of one theta_decompose_prelude call, following the
+    library's dispatch: one pipeline launch for bands of <= 4 layers; one
+    two-pass launch for longer bands whose rows for one CTA per SM fit the
+    kernel's 64 MB L2 budget (threads per row: the fewest of 32..256 giving
+    <= 4 vectors per thread within a 32 KB item); else a band-mean launch per
+    band and one row-pass launch."""
+    nmax = -(-L // G)
+    if nmax <= 4:
+        return 1
+    nv, row_bytes = I * b // 16, I * b
+    for cap in (4, 8):
+        tpr = next((t for t in (32, 64, 128, 256) if -(-nv // t) <= cap and (256 // t) * row_bytes <= 32 * 1024), None)
+        if tpr:
+            break
+    if tpr and nmax * (256 // tpr) * row_bytes * num_sms <= (64 << 20):
+        return 1
+    return G + 1
+
+
 def step_accounting(model=MODEL, r=RANK, m_values=M_VALUES, g_values=G_VALUES):
     """Per-stage algorithmic bytes / flops / kernel launches of one step."""
     L = model.num_layers
@@ -92,11 +112,8 @@ def step_accounting(model=MODEL, r=RANK, m_values=M_VALUES, g_values=G_VALUES):
                 fwd[m][0] += L * bytes_forward(m, O, I, r)
                 fwd[m][1] += L * flops_forward(m, O, I, r)
         nf = len(model.shapes)
-        # bands of <= 4 layers: one pipeline launch per family forms W0, s and R;
-        # longer bands: one band-mean launch per band, then one pipeline launch
-        one_pass = -(-L // G) <= 4
         stages.append(dict(name=f"prelude_G{G}", kind="prelude", bytes=pre, flops=0,
-                           launches=nf * (1 if one_pass else G + 1)))
+                           launches=sum(prelude_launches(L, G, I) for (_, I) in model.shapes.values())))
         stages.append(dict(name=f"reconstruct_G{G}", kind="reconstruct", bytes=rec, flops=0, launches=nf * L))
         stages.append(dict(name=f"frob_G{G}", kind="frob", bytes=fro, flops=0, launches=nf * L * 2))
         for m in m_values:
