@@ -189,8 +189,10 @@ int theta_frob_error(const void* original, const void* reconstructed, int64_t n,
  *              bytes (holds T = X . V); may be NULL when that size is 0.
  * THETA_BF16: tensor cores (tcgen05) with fp32 accumulation in tensor memory;
  * T = X.V is kept as a bf16 high part plus a bf16 low part, so the rank-r term
- * carries about 16 significand bits. THETA_F32: fp32 CUDA cores throughout.
- * rank == 0 allows U = V = NULL.
+ * carries about 16 significand bits. One or two tokens on a W0 of at most 32M
+ * elements take a CUDA-core sweep instead (fp32 accumulation, T in fp32).
+ * Grid sizing follows theta_set_policy. THETA_F32: fp32 CUDA cores
+ * throughout. rank == 0 allows U = V = NULL.
  */
 int theta_linear_forward(const void* X, int64_t M, int64_t I, const void* W0, int64_t O,
                          const float* s, const void* U, const void* V, int rank, theta_dtype dt,

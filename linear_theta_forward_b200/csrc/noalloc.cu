@@ -1,7 +1,9 @@
 // theta_linear_forward_noalloc: the theta forward with its scratch memory
 // built into the library instead of supplied by the caller.
 //
-// theta_linear_forward needs device scratch for T = X.V (4 * M * rank bytes).
+// theta_linear_forward needs device scratch for T = X.V: 4 * M * rank bytes
+// (the one- and two-token path keeps 16 fp32 partial sums of T instead,
+// 64 * M * rank bytes, at most 32 KB).
 // Most callers pass a buffer they allocated once. Some cannot allocate at
 // all: code that records a CUDA graph (cudaMalloc is not allowed while a
 // stream is being captured), engines whose device memory is handed out by
