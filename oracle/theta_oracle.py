@@ -178,6 +178,30 @@ def linear_forward(X, W0, s, U, V, out_dtype: str = "f64") -> np.ndarray:
     return round_to(Y, out_dtype)
 
 
+def gelu_tanh(x) -> np.ndarray:
+    """GELU in its tanh form, 0.5·x·(1 + tanh(√(2/π)·(x + 0.044715·x³))).
+
+    "Quality" — Native-equivalent at passthrough: the MLP takes its
+    activation from the model config, and Gemma 3 and Gemma 4 name gelu_tanh.
+    The formula is the published tanh approximation of GELU (Hendrycks and
+    Gimpel, 2016); the pages name the function, not the formula.
+    """
+    x = np.asarray(x, dtype=F64)
+    return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)))
+
+
+def gate_up_forward(X, gate, up, out_dtype: str = "f64") -> np.ndarray:
+    """Y = gelu_tanh(G) ⊙ P for an MLP's gate and up projections on the same
+    activations, each the theta forward of its own (W0, s, U, V): the product
+    that follows the two projections in the MLP ("Quality" — What quantizing
+    attention costs: the fused MLP). G and P are kept in fp64; the product is
+    rounded once.
+    """
+    G = linear_forward(X, *gate)
+    P = linear_forward(X, *up)
+    return round_to(gelu_tanh(G) * P, out_dtype)
+
+
 # -------------------------------------------------------- whole decomposition
 def decompose_family(weights, G: int, rank: int, dtype: str = "f64"):
     """Analytic decomposition of one projection family, in the pages' order:

@@ -317,6 +317,48 @@ def check_frob_statistics(o):
     assert 0.9 * expect < float(np.mean(errs)) <= expect * 1.01
 
 
-ALL_CHECKS = [check_round, check_bands, check_band_mean, check_row_scale, check_residual,
+def check_gelu(o):
+    """gelu_tanh: torch's tanh-form GELU, the odd-part identity
+    gelu(x) - gelu(-x) = x, its limits, and closeness to the erf form."""
+    import torch
+    from scipy.special import erf
+    x = np.linspace(-8.0, 8.0, 4001)
+    g = o.gelu_tanh(x)
+    ref = torch.nn.functional.gelu(torch.from_numpy(x), approximate="tanh").numpy()
+    assert np.allclose(g, ref, rtol=1e-12, atol=1e-13)
+    assert np.allclose(g - o.gelu_tanh(-x), x, rtol=0, atol=1e-12)
+    assert o.gelu_tanh(np.array([0.0]))[0] == 0.0
+    assert abs(o.gelu_tanh(np.array([30.0]))[0] - 30.0) < 1e-12
+    assert abs(o.gelu_tanh(np.array([-30.0]))[0]) < 1e-12
+    exact = 0.5 * x * (1.0 + erf(x / np.sqrt(2.0)))
+    assert np.max(np.abs(g - exact)) < 1e-3  # the approximation's known accuracy
+    assert np.max(np.abs(g - exact)) > 1e-5  # ... and it is the tanh form, not the erf one
+
+
+def check_gate_up(o):
+    """gate_up_forward against loops over the explicitly rebuilt weights and
+    torch's tanh-form GELU: gelu(X·W_gateᵀ) ⊙ (X·W_upᵀ)."""
+    import torch
+    rng = _rng(11)
+    M, O, I, r = 3, 4, 5, 2
+    X = rng.standard_normal((M, I))
+    gate = (rng.standard_normal((O, I)), rng.standard_normal(O), rng.standard_normal((O, r)),
+            rng.standard_normal((I, r)))
+    up = (rng.standard_normal((O, I)), rng.standard_normal(O), rng.standard_normal((O, r)),
+          rng.standard_normal((I, r)))
+    Y = o.gate_up_forward(X, gate, up)
+    Wg = np.diag(gate[1]) @ gate[0] + gate[2] @ gate[3].T
+    Wu = np.diag(up[1]) @ up[0] + up[2] @ up[3].T
+    for m in range(M):
+        for n in range(O):
+            g = sum(X[m, k] * Wg[n, k] for k in range(I))
+            u = sum(X[m, k] * Wu[n, k] for k in range(I))
+            act = torch.nn.functional.gelu(torch.tensor(g, dtype=torch.float64), approximate="tanh").item()
+            assert math.isclose(Y[m, n], act * u, rel_tol=1e-12, abs_tol=1e-12)
+    # the activation applies to the gate only: swapping the roles changes Y
+    assert not np.allclose(Y, o.gate_up_forward(X, up, gate))
+
+
+ALL_CHECKS = [check_gelu, check_gate_up, check_round, check_bands, check_band_mean, check_row_scale, check_residual,
               check_reconstruct, check_frob, check_forward, check_svd, check_decompose,
               check_frob_statistics]

@@ -121,7 +121,31 @@ def _m_svd_no_sigma(R, rank):
     return Uf[:, :rank], Vt[:rank].T
 
 
+def _m_gelu_erf(x):
+    from scipy.special import erf
+    x = np.asarray(x, np.float64)
+    return 0.5 * x * (1.0 + erf(x / np.sqrt(2.0)))
+
+
+def _m_gelu_constant(x):
+    x = np.asarray(x, np.float64)
+    return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.0447 * x ** 3)))
+
+
+def _m_gate_up_activates_up(X, gate, up, out_dtype="f64"):
+    return oracle.round_to(oracle.linear_forward(X, *gate) * oracle.gelu_tanh(oracle.linear_forward(X, *up)),
+                           out_dtype)
+
+
+def _m_gate_up_no_activation(X, gate, up, out_dtype="f64"):
+    return oracle.round_to(oracle.linear_forward(X, *gate) * oracle.linear_forward(X, *up), out_dtype)
+
+
 MUTANTS = {
+    "gelu_erf_form": dict(gelu_tanh=_m_gelu_erf),
+    "gelu_wrong_constant": dict(gelu_tanh=_m_gelu_constant),
+    "gate_up_activates_up": dict(gate_up_forward=_m_gate_up_activates_up),
+    "gate_up_without_activation": dict(gate_up_forward=_m_gate_up_no_activation),
     "round_truncates": dict(round_to=_m_round_truncate),
     "bands_late_remainder": dict(band_sizes=_m_bands_late_remainder),
     "bands_first_takes_all": dict(band_sizes=_m_bands_first_takes_all),
