@@ -627,6 +627,28 @@ def run_op(args):
             turn[0] += 1
             theta.theta_linear_forward(X, W0, s, U, V, Y, ws)
         nbytes, nflops = bytes_forward(M, O, I, r), flops_forward(M, O, I, r)
+    elif args.op == "gate_up":
+        nbuf = args.bufs if args.b2b else 1
+        X = syn.device_normal((M, I), 1.0, seed, "X", M, I)
+
+        def proj(k, tag):
+            return (syn.device_normal((O, I), 0.02, seed + k, "W0", tag, O, I),
+                    1.0 + syn.device_normal((O,), 0.05, seed + k, "s", tag, O, dtype="f32"),
+                    syn.device_normal((O, r), 0.01, seed + k, "U", tag, O, r) if r else None,
+                    syn.device_normal((I, r), 0.01, seed + k, "V", tag, I, r) if r else None)
+        probs = [(proj(k, "gate"), proj(k, "up"), torch.empty(M, O, dtype=torch.bfloat16, device="cuda"))
+                 for k in range(nbuf)]
+        nb = theta.theta_workspace_size(theta.THETA_OP_GATE_UP_FORWARD, M, O, I, r, theta.THETA_BF16)
+        ws = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
+        turn = [0]
+
+        def call():
+            gate, up, Y = probs[turn[0] % nbuf]
+            turn[0] += 1
+            theta.theta_linear_gate_up_forward(X, gate, up, Y, ws)
+        # both weights streamed once, X read once, one output written
+        nbytes = 2 * bytes_forward(M, O, I, r) - M * I * BF16 - M * O * BF16
+        nflops = 2 * flops_forward(M, O, I, r)
     elif args.op == "reconstruct":
         W0 = syn.device_normal((O, I), 0.02, seed, "W0", O, I)
         s = 1.0 + syn.device_normal((O,), 0.05, seed, "s", O, dtype="f32")
@@ -668,7 +690,7 @@ def run_op(args):
         torch.cuda.synchronize()
         ms = a.elapsed_time(b) / args.iters
         l2 = "calls back to back, no flush (mean of %d)" % args.iters
-        if args.op == "forward":
+        if args.op in ("forward", "gate_up"):
             l2 += ", cycling over %d independent problems" % args.bufs
     else:
         times = []
@@ -708,7 +730,7 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-rows", type=int, default=32)
-    ap.add_argument("--op", choices=["forward", "reconstruct", "prelude", "frob"],
+    ap.add_argument("--op", choices=["forward", "gate_up", "reconstruct", "prelude", "frob"],
                     help="time one entry point on one problem instead of the whole step")
     ap.add_argument("--M", type=int, default=256)
     ap.add_argument("--O", type=int, default=21504)

@@ -63,7 +63,8 @@ typedef enum { THETA_F32 = 0, THETA_BF16 = 1 } theta_dtype;
 
 typedef enum {
   THETA_OP_FROB_ERROR = 0,
-  THETA_OP_LINEAR_FORWARD = 1
+  THETA_OP_LINEAR_FORWARD = 1,
+  THETA_OP_GATE_UP_FORWARD = 2
 } theta_op;
 
 /* How the tensor-core kernels size their grids (see theta_set_policy). */
@@ -197,6 +198,35 @@ int theta_frob_error(const void* original, const void* reconstructed, int64_t n,
 int theta_linear_forward(const void* X, int64_t M, int64_t I, const void* W0, int64_t O,
                          const float* s, const void* U, const void* V, int rank, theta_dtype dt,
                          void* Y, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * theta_linear_gate_up_forward -- an MLP's gate and up projections of one
+ * layer, fused:  Y = gelu_tanh(G) (.) P  with
+ *   G = s_gate (.) (X . W0_gate^T) + (X . V_gate) . U_gate^T   (the gate projection)
+ *   P = s_up   (.) (X . W0_up^T)   + (X . V_up)   . U_up^T     (the up projection)
+ *   gelu_tanh(x) = 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))),
+ * the activation the Gemma models name in their config ("Quality" --
+ * Native-equivalent at passthrough: the MLP takes its activation from the
+ * config, gelu_tanh for Gemma 3 and 4; the fused MLP of "Quality" -- What
+ * quantizing attention costs). Each weight is rebuilt as in
+ * theta_linear_forward and never formed; G and P stay in fp32 until the
+ * product is rounded once to bf16.
+ *
+ *   X [M, I]; W0_gate, W0_up [O, I]; s_gate, s_up fp32 [O]; U_gate, U_up
+ *   [O, rank]; V_gate, V_up [I, rank]; Y [M, O], written. The two
+ *   projections share O, I and rank.
+ *   workspace  device scratch of theta_workspace_size(THETA_OP_GATE_UP_FORWARD)
+ *              bytes (both T = X . V), NULL when that size is 0 (rank 0).
+ * THETA_BF16 only (THETA_ERR_UNSUPPORTED otherwise): one tensor-core kernel
+ * streams both W0 tiles against each X tile it loads, with four accumulators
+ * in tensor memory (gate and up, main and rank terms) and the activation in
+ * its epilogue. Same alignment rules and policy as theta_linear_forward.
+ */
+int theta_linear_gate_up_forward(const void* X, int64_t M, int64_t I, int64_t O, int rank, theta_dtype dt,
+                                 const void* W0_gate, const float* s_gate, const void* U_gate,
+                                 const void* V_gate, const void* W0_up, const float* s_up, const void* U_up,
+                                 const void* V_up, void* Y, void* workspace, size_t workspace_bytes,
+                                 void* stream);
 
 /*
  * theta_linear_forward_noalloc -- theta_linear_forward for callers that

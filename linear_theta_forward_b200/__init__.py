@@ -15,6 +15,7 @@ import numpy as np
 
 __all__ = [
     "ThetaError", "THETA_F32", "THETA_BF16", "THETA_OP_FROB_ERROR", "THETA_OP_LINEAR_FORWARD",
+    "THETA_OP_GATE_UP_FORWARD", "theta_linear_gate_up_forward",
     "THETA_MAX_LAYERS", "LIB_PATH", "lib",
     "theta_version", "theta_status_string", "theta_last_error", "theta_band_index",
     "theta_band_mean", "theta_row_scale", "theta_residual", "theta_decompose_prelude",
@@ -26,7 +27,7 @@ __all__ = [
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtheta.so")
 
 THETA_F32, THETA_BF16 = 0, 1
-THETA_OP_FROB_ERROR, THETA_OP_LINEAR_FORWARD = 0, 1
+THETA_OP_FROB_ERROR, THETA_OP_LINEAR_FORWARD, THETA_OP_GATE_UP_FORWARD = 0, 1, 2
 THETA_POLICY_LATENCY, THETA_POLICY_THROUGHPUT = 0, 1
 THETA_MAX_LAYERS = 256
 
@@ -52,6 +53,8 @@ _SIGNATURES = {
     "theta_frob_error": (_int, _vp, _vp, _i64, _int, _vp, _vp, _sz, _vp),
     "theta_linear_forward": (_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp, _sz, _vp),
     "theta_linear_forward_noalloc": (_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp),
+    "theta_linear_gate_up_forward": (_int, _vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                     _vp, _vp, _sz, _vp),
     "theta_workspace_size": (_int, _int, _i64, _i64, _i64, _int, _int, ctypes.POINTER(_sz)),
     "theta_device_status": (_int, _vp),
 }
@@ -232,6 +235,24 @@ def theta_linear_forward(X, W0, s, U, V, Y, workspace=None, stream=None) -> None
                                     _ptr(U, "U", optional=True), _ptr(V, "V", optional=True), rank,
                                     _dtype_code(X), _ptr(Y, "Y"), ws_ptr, ws_bytes, _stream(stream)),
            "theta_linear_forward")
+
+
+def theta_linear_gate_up_forward(X, gate, up, Y, workspace=None, stream=None) -> None:
+    """Y [M, O] = gelu_tanh(gate projection) * (up projection), each a theta
+    forward on X; gate and up are (W0, s, U, V) tuples (U = V = None at rank
+    0). workspace: CUDA tensor of at least theta_workspace_size(
+    THETA_OP_GATE_UP_FORWARD, ...) bytes (None if 0)."""
+    M, I = X.shape
+    (W0g, sg, Ug, Vg), (W0u, su, Uu, Vu) = gate, up
+    O = W0g.shape[0]
+    rank = 0 if Ug is None else Ug.shape[1]
+    ws_ptr = _ptr(workspace, "workspace", optional=True)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_load().theta_linear_gate_up_forward(
+        _ptr(X, "X"), M, I, O, rank, _dtype_code(X), _ptr(W0g, "W0_gate"), _ptr(sg, "s_gate"),
+        _ptr(Ug, "U_gate", optional=True), _ptr(Vg, "V_gate", optional=True), _ptr(W0u, "W0_up"), _ptr(su, "s_up"),
+        _ptr(Uu, "U_up", optional=True), _ptr(Vu, "V_up", optional=True), _ptr(Y, "Y"), ws_ptr, ws_bytes,
+        _stream(stream)), "theta_linear_gate_up_forward")
 
 
 def theta_linear_forward_noalloc(X, W0, s, U, V, Y, stream=None) -> None:

@@ -68,6 +68,12 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
                         void* Y, void* ws, cudaError_t* cuda_err);
 // One bounded wait that nothing completes (gives up after limit_ms).
 cudaError_t launch_wait_selftest(const LaunchCtx& c, unsigned limit_ms);
+// Fused gate/up: Y = gelu_tanh(gate forward) * (up forward), one tile kernel
+// after the two T = X.V kernels.
+size_t gate_up_umma_workspace_bytes(int64_t M, int r);
+int launch_gate_up_umma(const LaunchCtx& c, const void* X, const void* W0g, const float* sg, const void* Ug,
+                        const void* Vg, const void* W0u, const float* su, const void* Uu, const void* Vu, int64_t M,
+                        int64_t O, int64_t I, int r, void* Y, void* ws, cudaError_t* ce);
 int launch_reconstruct_umma(const LaunchCtx& c, const float* s, const void* W0, const void* U,
                             const void* V, int64_t O, int64_t I, int r, void* W_out,
                             cudaError_t* cuda_err);

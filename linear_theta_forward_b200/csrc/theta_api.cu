@@ -310,6 +310,41 @@ THETA_API int theta_linear_forward(const void* X, int64_t M, int64_t I, const vo
   return THETA_OK;
 }
 
+THETA_API int theta_linear_gate_up_forward(const void* X, int64_t M, int64_t I, int64_t O, int rank,
+                                           theta_dtype dt, const void* W0_gate, const float* s_gate,
+                                           const void* U_gate, const void* V_gate, const void* W0_up,
+                                           const float* s_up, const void* U_up, const void* V_up, void* Y,
+                                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (!valid_dt(dt)) return fail(THETA_ERR_INVALID_ARG, "theta_linear_gate_up_forward: bad dtype %d", (int)dt);
+  if (M < 1 || I < 1 || O < 1 || rank < 0)
+    return fail(THETA_ERR_INVALID_ARG, "theta_linear_gate_up_forward: need M, I, O >= 1 and rank >= 0");
+  if (!X || !W0_gate || !s_gate || !W0_up || !s_up || !Y ||
+      (rank > 0 && (!U_gate || !V_gate || !U_up || !V_up)))
+    return fail(THETA_ERR_INVALID_ARG, "theta_linear_gate_up_forward: NULL pointer");
+  if (dt != THETA_BF16)
+    return fail(THETA_ERR_UNSUPPORTED, "theta_linear_gate_up_forward: bf16 only");
+  const size_t need = gate_up_umma_workspace_bytes(M, rank);
+  if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return fail(THETA_ERR_WORKSPACE, "theta_linear_gate_up_forward: need %zu bytes of 16-byte aligned workspace",
+                need);
+  for (const void* p : {X, W0_gate, W0_up, static_cast<const void*>(Y), static_cast<const void*>(s_gate),
+                        static_cast<const void*>(s_up)})
+    if (!aligned16(p))
+      return fail(THETA_ERR_ALIGNMENT, "theta_linear_gate_up_forward: bf16 needs 16-byte aligned pointers");
+  if ((rank > 0 && (!aligned16(U_gate) || !aligned16(V_gate) || !aligned16(U_up) || !aligned16(V_up))) || I % 8 ||
+      O % 8 || rank % 8)
+    return fail(THETA_ERR_ALIGNMENT,
+                "theta_linear_gate_up_forward: bf16 needs 16-byte aligned pointers and I, O, rank multiples of 8");
+  LaunchCtx c;
+  int st = make_ctx(stream, &c);
+  if (st) return st;
+  cudaError_t ce = cudaSuccess;
+  st = launch_gate_up_umma(c, X, W0_gate, s_gate, U_gate, V_gate, W0_up, s_up, U_up, V_up, M, O, I, rank, Y,
+                           workspace, &ce);
+  if (st == THETA_ERR_CUDA) return fail_cuda(ce, "theta_linear_gate_up_forward (tensor-core path)");
+  return st;
+}
+
 THETA_API int theta_workspace_size(int op, int64_t M, int64_t O, int64_t I, int rank, theta_dtype dt,
                                    size_t* bytes) {
   (void)O;
@@ -321,6 +356,10 @@ THETA_API int theta_workspace_size(int op, int64_t M, int64_t O, int64_t I, int 
     case THETA_OP_LINEAR_FORWARD:
       if (M < 1 || rank < 0) return fail(THETA_ERR_INVALID_ARG, "theta_workspace_size: bad M or rank");
       *bytes = forward_ws_bytes(M, rank, dt);
+      return THETA_OK;
+    case THETA_OP_GATE_UP_FORWARD:
+      if (M < 1 || rank < 0) return fail(THETA_ERR_INVALID_ARG, "theta_workspace_size: bad M or rank");
+      *bytes = gate_up_umma_workspace_bytes(M, rank);
       return THETA_OK;
   }
   return fail(THETA_ERR_INVALID_ARG, "theta_workspace_size: unknown op %d", op);

@@ -41,7 +41,7 @@ namespace theta {
 
 namespace {
 
-enum Mode { MODE_FORWARD = 0, MODE_XV = 1 };
+enum Mode { MODE_FORWARD = 0, MODE_XV = 1, MODE_GATE_UP = 2 };
 
 constexpr int kThreads = 192;
 constexpr int kBM = 128;       // MMA M (rows of A)
@@ -55,8 +55,9 @@ struct Args {
   int kb1;         // K blocks of phase 1
   int kb2;         // K blocks of phase 2 (0: none)
   int splits;      // cluster size along x (split-K)
-  const float* s;  // FORWARD row scale
-  bf16* out;       // FORWARD: Y [cols, rows]
+  const float* s;  // FORWARD row scale (GATE_UP: of the gate projection)
+  const float* s_up;  // GATE_UP: row scale of the up projection
+  bf16* out;       // FORWARD, GATE_UP: Y [cols, rows]
   bf16* t_hi;      // XV outputs [rows, r]
   bf16* t_lo;
   int r;
@@ -67,22 +68,38 @@ struct Args {
 template <int BN, int MODE>
 struct Cfg {
   static constexpr int kBBytes = BN * kBK * 2;  // XV: BN = padded rank, MN-major atoms of 64 columns
-  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kNumA = MODE == MODE_GATE_UP ? 2 : 1;  // A tiles per phase-1 stage
+  static constexpr int kStageBytes = kNumA * kABytes + kBBytes;
   // small rings for small BN so 2-3 decode CTAs share an SM
-  static constexpr int kStages = (BN == 128 || (MODE == MODE_XV && BN > 128)) ? 3 : 4;
-  static constexpr int kTmemNeed = MODE == MODE_FORWARD ? 2 * BN : BN;
+  // GATE_UP (two A tiles per stage): two CTAs per SM up to 64 tokens, a deep
+  // ring for the one CTA per SM of 128-token tiles
+  static constexpr int kStages = MODE == MODE_GATE_UP ? (BN == 128 ? 4 : BN == 64 ? 2 : 3)
+                                 : (BN == 128 || (MODE == MODE_XV && BN > 128)) ? 3 : 4;
+  // FORWARD: D1, D2; GATE_UP: D1 gate, D1 up, D2 gate, D2 up; XV: D1
+  static constexpr int kTmemNeed = MODE == MODE_FORWARD ? 2 * BN : MODE == MODE_GATE_UP ? 4 * BN : BN;
   static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
                                    : kTmemNeed <= 256 ? 256 : 512;
-  static constexpr int kPartialBytes = BN * kPitch * 4;
+  static_assert(kTmemNeed <= 512, "accumulators must fit in tensor memory");
+  // split-K partial tiles: one per output (GATE_UP: gate and up pre-activations)
+  static constexpr int kPartialBytes = kNumA * BN * kPitch * 4;
   static_assert(kPartialBytes <= kStages * kStageBytes, "partial tile must fit in the stage ring");
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
 };
+
+// GELU in its tanh form, the activation of the Gemma MLPs:
+// 0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))).
+__device__ __forceinline__ float gelu_tanh(float x) {
+  const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
+  return 0.5f * x * (1.f + tanhf(k0 * fmaf(0.044715f * x, x * x, x)));
+}
 
 template <int BN, int MODE>
 __global__ void __launch_bounds__(kThreads)
 umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
             const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-            const __grid_constant__ CUtensorMap tmB3, const Args args) {
+            const __grid_constant__ CUtensorMap tmB3, const __grid_constant__ CUtensorMap tmA1u,
+            const __grid_constant__ CUtensorMap tmA2u, const __grid_constant__ CUtensorMap tmB2u,
+            const __grid_constant__ CUtensorMap tmB3u, const Args args) {
   using C = Cfg<BN, MODE>;
   constexpr int S = C::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -100,9 +117,11 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
   const int m_tile = blockIdx.y;
   const int kb_begin = (int)((int64_t)split * args.kb1 / args.splits);
   const int kb_end = (int)((int64_t)(split + 1) * args.kb1 / args.splits);
-  const bool has_d2 = MODE == MODE_FORWARD && args.kb2 > 0 && split == 0;
+  constexpr bool kFwd = MODE == MODE_FORWARD || MODE == MODE_GATE_UP;
+  const bool has_d2 = kFwd && args.kb2 > 0 && split == 0;
   const int n1 = kb_end - kb_begin;
-  const int total = n1 + (has_d2 ? 2 * args.kb2 : 0);
+  // phase 2 items: (high, low) parts of T per projection
+  const int total = n1 + (has_d2 ? 2 * C::kNumA * args.kb2 : 0);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -129,7 +148,7 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
   // T = X.V kernel relies on exactly that: it starts early, streaming W0, X
   // and s at once (that kernel writes only T), and waits only before the
   // loads of T (the producer's rank phase) and in the epilogue.
-  const bool early = MODE == MODE_FORWARD && args.early_start;
+  const bool early = kFwd && args.early_start;
   if (!early) asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
@@ -151,11 +170,13 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
         break;
       }
       uint8_t* a = smem + st * C::kStageBytes;
-      uint8_t* b = a + kABytes;
-      ptx::mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+      uint8_t* b = a + C::kNumA * kABytes;
+      // phase 1 brings kNumA A tiles and the B tile; a phase-2 item one of each
+      ptx::mbar_arrive_expect_tx(&full[st], i < n1 ? C::kStageBytes : kABytes + C::kBBytes);
       if (i < n1) {
         const int kx = (kb_begin + i) * kBK;
         ptx::tma_load_2d(a, &tmA1, &full[st], kx, m_tile * kBM);
+        if constexpr (MODE == MODE_GATE_UP) ptx::tma_load_2d(a + kABytes, &tmA1u, &full[st], kx, m_tile * kBM);
         if constexpr (MODE == MODE_XV) {
           // V [I, r] row-major is MN-major for B: one box of 64 rank columns
           // x 64 rows of I per 64-wide column atom
@@ -168,8 +189,11 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
         const int j = i - n1;
         if (early && j == 0) asm volatile("griddepcontrol.wait;" ::: "memory");
         const int jx = (j % args.kb2) * kBK;
-        ptx::tma_load_2d(a, &tmA2, &full[st], jx, m_tile * kBM);
-        ptx::tma_load_2d(b, j < args.kb2 ? &tmB2 : &tmB3, &full[st], jx, n_tile * BN);
+        const int part = j / args.kb2;  // 0, 1: gate (or the forward) T high, low; 2, 3: up T high, low
+        const CUtensorMap* mA = part < 2 ? &tmA2 : &tmA2u;
+        const CUtensorMap* mB = part == 0 ? &tmB2 : part == 1 ? &tmB3 : part == 2 ? &tmB2u : &tmB3u;
+        ptx::tma_load_2d(a, mA, &full[st], jx, m_tile * kBM);
+        ptx::tma_load_2d(b, mB, &full[st], jx, n_tile * BN);
       }
       ++issued;
     }
@@ -196,22 +220,29 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
       }
       ptx::tc_fence_after();
       const uint32_t a = ptx::smem_u32(smem + st * C::kStageBytes);
-      const uint32_t b = a + kABytes;
+      const uint32_t b = a + C::kNumA * kABytes;
       if (i < n1) {
+        // tensor memory: D1 (GATE_UP: D1 gate at 0, D1 up at BN)
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
           const uint64_t ad = ptx::sdesc_sw128(a + kk * 32, 16, 1024);
           const uint64_t bd = MODE == MODE_XV ? ptx::sdesc_sw128(b + kk * 16 * 128, 64 * 128, 1024)
                                               : ptx::sdesc_sw128(b + kk * 32, 16, 1024);
           ptx::umma_bf16(tmem, ad, bd, idesc1, (i > 0 || kk > 0) ? 1u : 0u);
+          if constexpr (MODE == MODE_GATE_UP)
+            ptx::umma_bf16(tmem + BN, ptx::sdesc_sw128(a + kABytes + kk * 32, 16, 1024), bd, idesc1,
+                           (i > 0 || kk > 0) ? 1u : 0u);
         }
       } else {
+        // D2 after the D1 accumulators (GATE_UP: gate items first, then up)
         const int j = i - n1;
+        const int jd = j % (2 * args.kb2);  // item within its accumulator
+        const uint32_t d2 = tmem + (uint32_t)(C::kNumA * BN) + (uint32_t)(j / (2 * args.kb2)) * BN;
 #pragma unroll
         for (int kk = 0; kk < kBK / 16; ++kk) {
           const uint64_t ad = ptx::sdesc_sw128(a + kk * 32, 16, 1024);
           const uint64_t bd = ptx::sdesc_sw128(b + kk * 32, 16, 1024);
-          ptx::umma_bf16(tmem + BN, ad, bd, idesc2, (j > 0 || kk > 0) ? 1u : 0u);
+          ptx::umma_bf16(d2, ad, bd, idesc2, (jd > 0 || kk > 0) ? 1u : 0u);
         }
       }
       ptx::umma_commit(&empty[st]);
@@ -238,10 +269,36 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
     const int grow = m_tile * kBM + row;  // global row of A
     const int col0 = n_tile * BN;
     const int ncols = min(BN, args.cols - col0);
-    float so = 0.f;
-    if constexpr (MODE == MODE_FORWARD) so = (grow < args.rows) ? __ldg(args.s + grow) : 0.f;
+    float so = 0.f, su = 0.f;
+    if constexpr (kFwd) so = (grow < args.rows) ? __ldg(args.s + grow) : 0.f;
+    if constexpr (MODE == MODE_GATE_UP) su = (grow < args.rows) ? __ldg(args.s_up + grow) : 0.f;
     float* part = reinterpret_cast<float*>(smem);
-    if (ok) {
+    if (ok && MODE == MODE_GATE_UP) {
+      // gate g = s_g D1g + D2g and up u = s_u D1u + D2u; Y = gelu_tanh(g) u
+      for (int c0 = 0; c0 < ncols; c0 += 16) {
+        float g1[16], u1[16], g2[16], u2[16];
+        ptx::tmem_ld16(taddr + c0, g1);
+        ptx::tmem_ld16(taddr + BN + c0, u1);
+        if (has_d2) {
+          ptx::tmem_ld16(taddr + 2 * BN + c0, g2);
+          ptx::tmem_ld16(taddr + 3 * BN + c0, u2);
+        }
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float g = has_d2 ? fmaf(so, g1[e], g2[e]) : so * g1[e];
+          const float u = has_d2 ? fmaf(su, u1[e], u2[e]) : su * u1[e];
+          if (args.splits > 1) {
+            part[(c0 + e) * kPitch + row] = g;
+            part[(BN + c0 + e) * kPitch + row] = u;
+          } else {
+            const int m = col0 + c0 + e;
+            if (grow < args.rows && m < args.cols)
+              args.out[(int64_t)m * args.rows + grow] = __float2bfloat16_rn(gelu_tanh(g) * u);
+          }
+        }
+      }
+    } else if (ok) {
       for (int c0 = 0; c0 < ncols; c0 += 16) {
         float d1[16], d2[16];
         ptx::tmem_ld16(taddr + c0, d1);
@@ -299,6 +356,12 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
         if (grow >= args.rows) continue;
         if constexpr (MODE == MODE_FORWARD) {
           args.out[(int64_t)(col0 + c) * args.rows + grow] = __float2bfloat16_rn(v);
+        } else if constexpr (MODE == MODE_GATE_UP) {
+          // v is the gate pre-activation; the up one is the tile BN columns further
+          const uint32_t off_u = off + (uint32_t)(BN * kPitch * 4);
+          float u = 0.f;
+          for (int p = 0; p < args.splits; ++p) u += ptx::ld_dsmem_f32(ptx::mapa(off_u, (uint32_t)p));
+          args.out[(int64_t)(col0 + c) * args.rows + grow] = __float2bfloat16_rn(gelu_tanh(v) * u);
         } else if constexpr (MODE == MODE_XV) {
           const int j = col0 + c;
           if (j < args.r) {
@@ -587,9 +650,14 @@ int pick_splits(int64_t tiles, int kb, int capacity, int max_cluster) {
   return s;
 }
 
+// The tensor maps of one launch: A1, B1 (phase 1), A2, B2, B3 (phase 2), and
+// for GATE_UP the up projection's A1, A2, B2, B3 (other modes repeat A1).
+struct Maps {
+  CUtensorMap a1, b1, a2, b2, b3, a1u, a2u, b2u, b3u;
+};
+
 template <int BN, int MODE>
-cudaError_t launch_tile_kernel(const LaunchCtx& c, const CUtensorMap& a1, const CUtensorMap& b1, const CUtensorMap& a2,
-                               const CUtensorMap& b2, const CUtensorMap& b3, Args args, int m_tiles, int n_tiles) {
+cudaError_t launch_tile_kernel(const LaunchCtx& c, const Maps& mp, Args args, int m_tiles, int n_tiles) {
   using C = Cfg<BN, MODE>;
   auto kern = umma_kernel<BN, MODE>;
   static KernelInfo info[64];
@@ -605,7 +673,7 @@ cudaError_t launch_tile_kernel(const LaunchCtx& c, const CUtensorMap& a1, const 
                     ? 1
                     : pick_splits(tiles, args.kb1, capacity, info[c.device].max_cluster);
   return launch_pdl(kern, dim3((unsigned)(n_tiles * args.splits), (unsigned)m_tiles, 1), dim3(kThreads), C::kSmemBytes,
-                    c.stream, args.splits, a1, b1, a2, b2, b3, args);
+                    c.stream, args.splits, mp.a1, mp.b1, mp.a2, mp.b2, mp.b3, mp.a1u, mp.a2u, mp.b2u, mp.b3u, args);
 }
 
 template <int KB>
@@ -647,6 +715,42 @@ size_t forward_umma_workspace_bytes(int64_t M, int r) {
   return 2 * half > gemv ? 2 * half : gemv;
 }
 
+namespace {
+
+// T = X . V (fp32 in tensor memory) -> bf16 high and low parts [M, r]
+int launch_xv_umma(const LaunchCtx& c, const void* X, const void* V, int64_t M, int64_t I, int r, bf16* t_hi,
+                   bf16* t_lo, cudaError_t* ce) {
+  Maps mp;
+  int st;
+  if ((st = make_map(&mp.a1, X, M, I, kBM, ce))) return st;  // 128 token rows per tile
+  if ((st = make_map(&mp.b1, V, I, r, kBK, ce))) return st;  // box: 64 rank columns x 64 rows of I
+  mp.a2 = mp.b2 = mp.b3 = mp.a1u = mp.a2u = mp.b2u = mp.b3u = mp.b1;
+  Args a = {};
+  a.rows = (int)M;
+  a.cols = r;
+  a.kb1 = (int)ceil_div(I, kBK);
+  a.kb2 = 0;
+  a.t_hi = t_hi;
+  a.t_lo = t_lo;
+  a.r = r;
+  a.err = c.err;
+  const int m_tiles = (int)ceil_div(M, kBM);
+  cudaError_t e;
+  switch ((int)ceil_div(r, 64) * 64) {
+    case 64: e = launch_tile_kernel<64, MODE_XV>(c, mp, a, m_tiles, 1); break;
+    case 128: e = launch_tile_kernel<128, MODE_XV>(c, mp, a, m_tiles, 1); break;
+    case 192: e = launch_tile_kernel<192, MODE_XV>(c, mp, a, m_tiles, 1); break;
+    default: e = launch_tile_kernel<256, MODE_XV>(c, mp, a, m_tiles, 1); break;
+  }
+  if (e != cudaSuccess) {
+    *ce = e;
+    return THETA_ERR_CUDA;
+  }
+  return THETA_OK;
+}
+
+}  // namespace
+
 int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const float* s, const void* U,
                         const void* V, int64_t M, int64_t O, int64_t I, int r, void* Y, void* ws,
                         cudaError_t* ce) {
@@ -665,51 +769,29 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
   const int kb = (int)ceil_div(I, kBK);
   bf16* t_hi = nullptr;
   bf16* t_lo = nullptr;
-  CUtensorMap mX, mW0, mU, mThi, mTlo, mV;
   int st;
   if (r > 0) {
     t_hi = static_cast<bf16*>(ws);
     t_lo = reinterpret_cast<bf16*>(static_cast<uint8_t*>(ws) + forward_umma_workspace_bytes(M, r) / 2);
-    // ---- T = X . V (fp32 in tensor memory) -> bf16 high and low parts
-    if ((st = make_map(&mX, X, M, I, kBM, ce))) return st;  // 128 token rows per tile
-    if ((st = make_map(&mV, V, I, r, kBK, ce))) return st;  // box: 64 rank columns x 64 rows of I
-    Args a = {};
-    a.rows = (int)M;
-    a.cols = r;
-    a.kb1 = kb;
-    a.kb2 = 0;
-    a.t_hi = t_hi;
-    a.t_lo = t_lo;
-    a.r = r;
-    a.err = c.err;
-    const int m_tiles = (int)ceil_div(M, kBM);
-    const int rp = (int)ceil_div(r, 64) * 64;
-    switch (rp) {
-      case 64: e = launch_tile_kernel<64, MODE_XV>(c, mX, mV, mV, mV, mV, a, m_tiles, 1); break;
-      case 128: e = launch_tile_kernel<128, MODE_XV>(c, mX, mV, mV, mV, mV, a, m_tiles, 1); break;
-      case 192: e = launch_tile_kernel<192, MODE_XV>(c, mX, mV, mV, mV, mV, a, m_tiles, 1); break;
-      default: e = launch_tile_kernel<256, MODE_XV>(c, mX, mV, mV, mV, mV, a, m_tiles, 1); break;
-    }
-    if (e != cudaSuccess) {
-      *ce = e;
-      return THETA_ERR_CUDA;
-    }
+    if ((st = launch_xv_umma(c, X, V, M, I, r, t_hi, t_lo, ce))) return st;
   }
   // ---- Y = s * (X . W0^T) + T . U^T, swap-AB: W0 rows are the MMA M side
   const int BN = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 256 ? 128 : 256;
   const int m_tiles = (int)ceil_div(O, kBM);
   const int n_tiles = (int)ceil_div(M, BN);
-  if ((st = make_map(&mW0, W0, O, I, kBM, ce))) return st;
-  CUtensorMap mXb;
-  if ((st = make_map(&mXb, X, M, I, BN, ce))) return st;
+  Maps mp;
+  if ((st = make_map(&mp.a1, W0, O, I, kBM, ce))) return st;
+  if ((st = make_map(&mp.b1, X, M, I, BN, ce))) return st;
   if (r > 0) {
-    if ((st = make_map(&mU, U, O, r, kBM, ce))) return st;
-    if ((st = make_map(&mThi, t_hi, M, r, BN, ce))) return st;
-    if ((st = make_map(&mTlo, t_lo, M, r, BN, ce))) return st;
+    if ((st = make_map(&mp.a2, U, O, r, kBM, ce))) return st;
+    if ((st = make_map(&mp.b2, t_hi, M, r, BN, ce))) return st;
+    if ((st = make_map(&mp.b3, t_lo, M, r, BN, ce))) return st;
   } else {
-    mU = mW0;
-    mThi = mTlo = mXb;
+    mp.a2 = mp.a1;
+    mp.b2 = mp.b3 = mp.b1;
   }
+  mp.a1u = mp.a2u = mp.a1;
+  mp.b2u = mp.b3u = mp.b1;
   Args a = {};
   a.rows = (int)O;
   a.cols = (int)M;
@@ -720,11 +802,74 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
   a.early_start = r > 0;  // directly after this call's T = X.V kernel
   a.err = c.err;
   switch (BN) {
-    case 16: e = launch_tile_kernel<16, MODE_FORWARD>(c, mW0, mXb, mU, mThi, mTlo, a, m_tiles, n_tiles); break;
-    case 32: e = launch_tile_kernel<32, MODE_FORWARD>(c, mW0, mXb, mU, mThi, mTlo, a, m_tiles, n_tiles); break;
-    case 64: e = launch_tile_kernel<64, MODE_FORWARD>(c, mW0, mXb, mU, mThi, mTlo, a, m_tiles, n_tiles); break;
-    case 128: e = launch_tile_kernel<128, MODE_FORWARD>(c, mW0, mXb, mU, mThi, mTlo, a, m_tiles, n_tiles); break;
-    default: e = launch_tile_kernel<256, MODE_FORWARD>(c, mW0, mXb, mU, mThi, mTlo, a, m_tiles, n_tiles); break;
+    case 16: e = launch_tile_kernel<16, MODE_FORWARD>(c, mp, a, m_tiles, n_tiles); break;
+    case 32: e = launch_tile_kernel<32, MODE_FORWARD>(c, mp, a, m_tiles, n_tiles); break;
+    case 64: e = launch_tile_kernel<64, MODE_FORWARD>(c, mp, a, m_tiles, n_tiles); break;
+    case 128: e = launch_tile_kernel<128, MODE_FORWARD>(c, mp, a, m_tiles, n_tiles); break;
+    default: e = launch_tile_kernel<256, MODE_FORWARD>(c, mp, a, m_tiles, n_tiles); break;
+  }
+  if (e != cudaSuccess) {
+    *ce = e;
+    return THETA_ERR_CUDA;
+  }
+  return THETA_OK;
+}
+
+size_t gate_up_umma_workspace_bytes(int64_t M, int r) {
+  if (r <= 0) return 0;
+  const size_t half = ((size_t)M * r * 2 + 255) / 256 * 256;
+  return 4 * half;  // T high and low parts of the gate, then of the up projection
+}
+
+int launch_gate_up_umma(const LaunchCtx& c, const void* X, const void* W0g, const float* sg, const void* Ug,
+                        const void* Vg, const void* W0u, const float* su, const void* Uu, const void* Vu, int64_t M,
+                        int64_t O, int64_t I, int r, void* Y, void* ws, cudaError_t* ce) {
+  *ce = cudaSuccess;
+  if (O > (int64_t)65535 * kBM || M > ((int64_t)1 << 30) || I > ((int64_t)1 << 31) - 64 || r > 256)
+    return THETA_ERR_UNSUPPORTED;
+  const size_t half = ((size_t)M * r * 2 + 255) / 256 * 256;
+  bf16* t[4] = {};
+  int st;
+  if (r > 0) {
+    for (int q = 0; q < 4; ++q) t[q] = reinterpret_cast<bf16*>(static_cast<uint8_t*>(ws) + q * half);
+    if ((st = launch_xv_umma(c, X, Vg, M, I, r, t[0], t[1], ce))) return st;
+    if ((st = launch_xv_umma(c, X, Vu, M, I, r, t[2], t[3], ce))) return st;
+  }
+  // four accumulators of BN columns: at most 128 tokens per tile
+  const int BN = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  const int m_tiles = (int)ceil_div(O, kBM);
+  const int n_tiles = (int)ceil_div(M, BN);
+  Maps mp;
+  if ((st = make_map(&mp.a1, W0g, O, I, kBM, ce))) return st;
+  if ((st = make_map(&mp.a1u, W0u, O, I, kBM, ce))) return st;
+  if ((st = make_map(&mp.b1, X, M, I, BN, ce))) return st;
+  if (r > 0) {
+    if ((st = make_map(&mp.a2, Ug, O, r, kBM, ce))) return st;
+    if ((st = make_map(&mp.b2, t[0], M, r, BN, ce))) return st;
+    if ((st = make_map(&mp.b3, t[1], M, r, BN, ce))) return st;
+    if ((st = make_map(&mp.a2u, Uu, O, r, kBM, ce))) return st;
+    if ((st = make_map(&mp.b2u, t[2], M, r, BN, ce))) return st;
+    if ((st = make_map(&mp.b3u, t[3], M, r, BN, ce))) return st;
+  } else {
+    mp.a2 = mp.a2u = mp.a1;
+    mp.b2 = mp.b3 = mp.b2u = mp.b3u = mp.b1;
+  }
+  Args a = {};
+  a.rows = (int)O;
+  a.cols = (int)M;
+  a.kb1 = (int)ceil_div(I, kBK);
+  a.kb2 = r > 0 ? (int)ceil_div(r, kBK) : 0;
+  a.s = sg;
+  a.s_up = su;
+  a.out = static_cast<bf16*>(Y);
+  a.early_start = r > 0;  // directly after the up projection's T = X.V kernel
+  a.err = c.err;
+  cudaError_t e;
+  switch (BN) {
+    case 16: e = launch_tile_kernel<16, MODE_GATE_UP>(c, mp, a, m_tiles, n_tiles); break;
+    case 32: e = launch_tile_kernel<32, MODE_GATE_UP>(c, mp, a, m_tiles, n_tiles); break;
+    case 64: e = launch_tile_kernel<64, MODE_GATE_UP>(c, mp, a, m_tiles, n_tiles); break;
+    default: e = launch_tile_kernel<128, MODE_GATE_UP>(c, mp, a, m_tiles, n_tiles); break;
   }
   if (e != cudaSuccess) {
     *ce = e;

@@ -87,6 +87,23 @@ def test_validation_happens_before_any_cuda_call(lib):
     assert raw.theta_linear_forward(ctypes.c_void_p(16), 4, 8, ctypes.c_void_p(16), 8, ctypes.c_void_p(16),
                                     ctypes.c_void_p(16), ctypes.c_void_p(16), 8, 1, ctypes.c_void_p(16),
                                     None, 0, None) == -6                                         # no workspace
+    p = ctypes.c_void_p(16)
+    assert raw.theta_linear_gate_up_forward(None, 4, 8, 8, 0, 1, None, None, None, None, None, None, None, None,
+                                            None, None, 0, None) == -1                           # NULL inputs
+    assert raw.theta_linear_gate_up_forward(p, 4, 8, 8, 8, 0, p, p, p, p, p, p, p, p, p, p, 1 << 20,
+                                            None) == -2                                          # fp32: bf16 only
+    assert raw.theta_linear_gate_up_forward(p, 4, 8, 8, 8, 1, p, p, p, p, p, p, p, p, p, None, 0,
+                                            None) == -6                                          # no workspace
+    assert raw.theta_linear_gate_up_forward(p, 4, 12, 8, 8, 1, p, p, p, p, p, p, p, p, p, p, 1 << 20,
+                                            None) == -3                                          # I % 8 != 0
+
+
+def test_gate_up_workspace_covers_both_projections(lib):
+    for M, r in [(1, 8), (16, 32), (300, 64)]:
+        one = lib.theta_workspace_size(lib.THETA_OP_LINEAR_FORWARD, M, 64, 64, r, lib.THETA_BF16)
+        both = lib.theta_workspace_size(lib.THETA_OP_GATE_UP_FORWARD, M, 64, 64, r, lib.THETA_BF16)
+        assert both >= 4 * M * r * 2 and both % 256 == 0 and both >= 2 * min(one, 4 * M * r * 2)
+    assert lib.theta_workspace_size(lib.THETA_OP_GATE_UP_FORWARD, 16, 64, 64, 0, lib.THETA_BF16) == 0
 
 
 def test_workspace_sizes(lib):
