@@ -140,6 +140,32 @@ def truncated_svd(R, rank: int):
     return Uf[:, :rank] * sig[:rank], Vt[:rank].T.copy()
 
 
+def randomized_svd(R, rank: int, omega, power_iters: int = 0):
+    """Rank-r factors of a large residual by the randomized algorithm the pages
+    name ("The theta bundle" -- Low-rank residual: Halko et al., 2009, for
+    large matrices; U absorbs the singular values). The steps follow Halko,
+    Martinsson and Tropp: sample the range, Y = R·Ωᵀ, and orthonormalize it
+    (Q); optionally refine by subspace iteration (Q ← orth(R·orth(Rᵀ·Q)),
+    power_iters times); project, B = Qᵀ·R; take the SVD of the small B; and
+    lift back, U = Q·Ũ[:, :r]·diag(σ[:r]), V = W[:, :r].
+
+    omega [k, I] holds the Gaussian test matrix (k = r + oversampling), passed
+    in so that the GPU and this function see the same draw. Returns
+    (U [O, r], V [I, r]).
+    """
+    Rm = np.asarray(R, dtype=F64)
+    Om = np.asarray(omega, dtype=F64)
+    if rank == 0:
+        return np.zeros((Rm.shape[0], 0)), np.zeros((Rm.shape[1], 0))
+    Q, _ = np.linalg.qr(Rm @ Om.T)
+    for _ in range(power_iters):
+        Z, _ = np.linalg.qr(Rm.T @ Q)
+        Q, _ = np.linalg.qr(Rm @ Z)
+    B = Q.T @ Rm
+    Ub, sig, Wt = np.linalg.svd(B, full_matrices=False)
+    return (Q @ Ub[:, :rank]) * sig[:rank], Wt[:rank].T.copy()
+
+
 def reconstruct(s, W0, U, V, out_dtype: str = "f64") -> np.ndarray:
     """reconstruct_weight(s, W0, U, V) = diag(s)·W0 + U·Vᵀ
     ("The theta bundle" -- the approximation formula and Key layout)."""

@@ -280,7 +280,42 @@ def check_svd(o):
     assert np.allclose(U @ V.T, R, atol=1e-12)
 
 
-# --------------------------------------------------------------- pipeline
+def check_randomized_svd(o):
+    """randomized_svd: exact on matrices of rank <= r; with a square test
+    matrix (k = min(O, I)) it is the truncated SVD, so Eckart-Young fixes its
+    error; on a decaying spectrum two subspace iterations land within 1% of
+    the optimum; V is orthonormal and U's column norms are B's singular
+    values; rank 0 gives empty factors."""
+    rng = _rng(21)
+    O, I, r = 40, 30, 5
+    # exact rank r: recovered to rounding whatever the draw
+    R = rng.standard_normal((O, r)) @ rng.standard_normal((r, I))
+    omega = rng.standard_normal((r + 4, I))
+    U, V = o.randomized_svd(R, r, omega)
+    assert U.shape == (O, r) and V.shape == (I, r)
+    assert np.allclose(U @ V.T, R, atol=1e-10 * np.abs(R).max())
+    # k = I: the sample spans everything, so the result is the truncated SVD
+    R = rng.standard_normal((O, I))
+    eig = np.sort(np.linalg.eigvalsh(R.T @ R))[::-1]
+    U, V = o.randomized_svd(R, r, rng.standard_normal((I, I)))
+    err2 = np.sum((R - U @ V.T) ** 2)
+    assert math.isclose(err2, float(np.sum(eig[r:])), rel_tol=1e-9)
+    assert np.allclose(V.T @ V, np.eye(r), atol=1e-12)
+    assert np.allclose(np.sum(U ** 2, axis=0), eig[:r], rtol=1e-9)
+    # decaying spectrum, k = r + 6, two power iterations: near-optimal
+    A, _ = np.linalg.qr(rng.standard_normal((O, I)))
+    Bq, _ = np.linalg.qr(rng.standard_normal((I, I)))
+    sig = 0.7 ** np.arange(I)
+    R = (A * sig) @ Bq.T
+    U, V = o.randomized_svd(R, r, rng.standard_normal((r + 6, I)), power_iters=2)
+    opt = float(np.sum(sig[r:] ** 2))
+    err2 = float(np.sum((R - U @ V.T) ** 2))
+    assert opt <= err2 * (1 + 1e-9) and err2 <= 1.01 * opt
+    U0, V0 = o.randomized_svd(R, 0, rng.standard_normal((4, I)))
+    assert U0.shape == (O, 0) and V0.shape == (I, 0)
+
+
+# --------------------------------------------------------------- pipeline# --------------------------------------------------------------- pipeline
 def check_decompose(o):
     rng = _rng(9)
     L, O, I = 4, 6, 10
@@ -359,6 +394,6 @@ def check_gate_up(o):
     assert not np.allclose(Y, o.gate_up_forward(X, up, gate))
 
 
-ALL_CHECKS = [check_gelu, check_gate_up, check_round, check_bands, check_band_mean, check_row_scale, check_residual,
+ALL_CHECKS = [check_gelu, check_gate_up, check_randomized_svd, check_round, check_bands, check_band_mean, check_row_scale, check_residual,
               check_reconstruct, check_frob, check_forward, check_svd, check_decompose,
               check_frob_statistics]

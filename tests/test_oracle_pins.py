@@ -141,7 +141,22 @@ def _m_gate_up_no_activation(X, gate, up, out_dtype="f64"):
     return oracle.round_to(oracle.linear_forward(X, *gate) * oracle.linear_forward(X, *up), out_dtype)
 
 
+def _m_rsvd_unorthonormalized(R, rank, omega, power_iters=0):
+    Rm, Om = np.asarray(R, np.float64), np.asarray(omega, np.float64)
+    Q = Rm @ Om.T  # the sample used as if it were an orthonormal basis
+    Ub, sig, Wt = np.linalg.svd(Q.T @ Rm, full_matrices=False)
+    return (Q @ Ub[:, :rank]) * sig[:rank], Wt[:rank].T.copy()
+
+
+def _m_rsvd_sigma_in_v(R, rank, omega, power_iters=0):
+    U, V = oracle.randomized_svd(R, rank, omega, power_iters)
+    n = np.linalg.norm(U, axis=0)
+    return U / np.where(n == 0, 1, n), V * n
+
+
 MUTANTS = {
+    "rsvd_sample_not_orthonormalized": dict(randomized_svd=_m_rsvd_unorthonormalized),
+    "rsvd_sigma_in_v": dict(randomized_svd=_m_rsvd_sigma_in_v),
     "gelu_erf_form": dict(gelu_tanh=_m_gelu_erf),
     "gelu_wrong_constant": dict(gelu_tanh=_m_gelu_constant),
     "gate_up_activates_up": dict(gate_up_forward=_m_gate_up_activates_up),
