@@ -649,6 +649,18 @@ def run_op(args):
         # both weights streamed once, X read once, one output written
         nbytes = 2 * bytes_forward(M, O, I, r) - M * I * BF16 - M * O * BF16
         nflops = 2 * flops_forward(M, O, I, r)
+    elif args.op == "svd":
+        # randomized SVD of one residual: rank r, r + 10 samples, 2 subspace iterations
+        k, q = min(r + 10, O, I), 2
+        R = syn.device_normal((O, I), 0.005, seed, "R", O, I)
+        omega = syn.device_normal((k, I), 1.0, seed, "omega", k, I, dtype="f32")
+        Ud = torch.empty(O, r, dtype=torch.bfloat16, device="cuda")
+        Vd = torch.empty(I, r, dtype=torch.bfloat16, device="cuda")
+        ws = torch.empty(theta.theta_workspace_size(theta.THETA_OP_RESIDUAL_SVD, k, O, I, r, theta.THETA_BF16),
+                         dtype=torch.uint8, device="cuda")
+        call = lambda: theta.theta_residual_svd(R, r, omega, Ud, Vd, ws, power_iters=q)  # noqa: E731
+        # R is read by 2 + 2q products (R.Omega^T, 2 per iteration, Q^T.R)
+        nbytes, nflops = (2 + 2 * q) * O * I * BF16, (2 + 2 * q) * 2 * O * I * k
     elif args.op == "reconstruct":
         W0 = syn.device_normal((O, I), 0.02, seed, "W0", O, I)
         s = 1.0 + syn.device_normal((O,), 0.05, seed, "s", O, dtype="f32")
@@ -730,7 +742,7 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-rows", type=int, default=32)
-    ap.add_argument("--op", choices=["forward", "gate_up", "reconstruct", "prelude", "frob"],
+    ap.add_argument("--op", choices=["forward", "gate_up", "reconstruct", "prelude", "frob", "svd"],
                     help="time one entry point on one problem instead of the whole step")
     ap.add_argument("--M", type=int, default=256)
     ap.add_argument("--O", type=int, default=21504)

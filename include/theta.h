@@ -64,7 +64,8 @@ typedef enum { THETA_F32 = 0, THETA_BF16 = 1 } theta_dtype;
 typedef enum {
   THETA_OP_FROB_ERROR = 0,
   THETA_OP_LINEAR_FORWARD = 1,
-  THETA_OP_GATE_UP_FORWARD = 2
+  THETA_OP_GATE_UP_FORWARD = 2,
+  THETA_OP_RESIDUAL_SVD = 3
 } theta_op;
 
 /* How the tensor-core kernels size their grids (see theta_set_policy). */
@@ -151,6 +152,29 @@ int theta_residual(const void* weight, const void* W0, const float* s, int64_t O
 int theta_decompose_prelude(const void* const* weights, int num_layers, int G, int64_t O,
                             int64_t I, theta_dtype dt, void* const* W0, float* const* s,
                             void* const* residual, void* stream);
+
+/*
+ * theta_residual_svd -- rank-r factors of a residual, U . V^T ~ R, with U
+ * absorbing the singular values ("The theta bundle" -- Low-rank residual:
+ * a randomized SVD, Halko et al., for large matrices). Steps: range sample
+ * Y = R . omega^T; orthonormal basis Q of Y (shifted Cholesky QR, then two
+ * plain passes); power_iters rounds of subspace iteration; B = Q^T . R; the
+ * eigen-decomposition of B . B^T (Jacobi, fp64) gives B's singular vectors;
+ * U = Q . E_r . diag(sigma), V = B^T . E_r . diag(1 / sigma).
+ *
+ *   R [O, I] (dt); omega fp32 [samples, I], the Gaussian test matrix (the
+ *   caller draws it; samples = rank + oversampling); U [O, rank] and
+ *   V [I, rank] (dt), written. 1 <= rank <= samples <= min(96, O, I);
+ *   0 <= power_iters <= 8.
+ *   workspace  device scratch of theta_workspace_size(THETA_OP_RESIDUAL_SVD,
+ *              samples, O, I, rank, dt) bytes (M carries samples).
+ * fp32 arithmetic on CUDA cores (fp64 for the k x k steps): decomposition
+ * work, not the projection's hot path. A direction the sample lacks (R of
+ * rank below samples) comes out as a zero column of U and V.
+ */
+int theta_residual_svd(const void* R, int64_t O, int64_t I, theta_dtype dt, int rank, int samples,
+                       int power_iters, const float* omega, void* U, void* V, void* workspace,
+                       size_t workspace_bytes, void* stream);
 
 /*
  * theta_reconstruct -- reconstruct_weight(s, W0, U, V) = diag(s) . W0 + U . V^T

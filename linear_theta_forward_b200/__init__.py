@@ -15,7 +15,7 @@ import numpy as np
 
 __all__ = [
     "ThetaError", "THETA_F32", "THETA_BF16", "THETA_OP_FROB_ERROR", "THETA_OP_LINEAR_FORWARD",
-    "THETA_OP_GATE_UP_FORWARD", "theta_linear_gate_up_forward",
+    "THETA_OP_GATE_UP_FORWARD", "theta_linear_gate_up_forward", "THETA_OP_RESIDUAL_SVD", "theta_residual_svd",
     "THETA_MAX_LAYERS", "LIB_PATH", "lib",
     "theta_version", "theta_status_string", "theta_last_error", "theta_band_index",
     "theta_band_mean", "theta_row_scale", "theta_residual", "theta_decompose_prelude",
@@ -27,7 +27,7 @@ __all__ = [
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtheta.so")
 
 THETA_F32, THETA_BF16 = 0, 1
-THETA_OP_FROB_ERROR, THETA_OP_LINEAR_FORWARD, THETA_OP_GATE_UP_FORWARD = 0, 1, 2
+THETA_OP_FROB_ERROR, THETA_OP_LINEAR_FORWARD, THETA_OP_GATE_UP_FORWARD, THETA_OP_RESIDUAL_SVD = 0, 1, 2, 3
 THETA_POLICY_LATENCY, THETA_POLICY_THROUGHPUT = 0, 1
 THETA_MAX_LAYERS = 256
 
@@ -53,6 +53,7 @@ _SIGNATURES = {
     "theta_frob_error": (_int, _vp, _vp, _i64, _int, _vp, _vp, _sz, _vp),
     "theta_linear_forward": (_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp, _sz, _vp),
     "theta_linear_forward_noalloc": (_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp),
+    "theta_residual_svd": (_int, _vp, _i64, _i64, _int, _int, _int, _int, _vp, _vp, _vp, _vp, _sz, _vp),
     "theta_linear_gate_up_forward": (_int, _vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                      _vp, _vp, _sz, _vp),
     "theta_workspace_size": (_int, _int, _i64, _i64, _i64, _int, _int, ctypes.POINTER(_sz)),
@@ -253,6 +254,18 @@ def theta_linear_gate_up_forward(X, gate, up, Y, workspace=None, stream=None) ->
         _ptr(Ug, "U_gate", optional=True), _ptr(Vg, "V_gate", optional=True), _ptr(W0u, "W0_up"), _ptr(su, "s_up"),
         _ptr(Uu, "U_up", optional=True), _ptr(Vu, "V_up", optional=True), _ptr(Y, "Y"), ws_ptr, ws_bytes,
         _stream(stream)), "theta_linear_gate_up_forward")
+
+
+def theta_residual_svd(R, rank, omega, U, V, workspace, power_iters=2, stream=None) -> None:
+    """U [O, rank], V [I, rank] with U·Vᵀ ≈ R by the randomized SVD; omega is
+    the fp32 Gaussian test matrix [samples, I]; workspace: CUDA tensor of at
+    least theta_workspace_size(THETA_OP_RESIDUAL_SVD, samples, O, I, rank) bytes."""
+    O, I = R.shape
+    samples = omega.shape[0]
+    _check(_load().theta_residual_svd(_ptr(R, "R"), O, I, _dtype_code(R), int(rank), int(samples), int(power_iters),
+                                      _ptr(omega, "omega"), _ptr(U, "U"), _ptr(V, "V"), _ptr(workspace, "workspace"),
+                                      workspace.numel() * workspace.element_size(), _stream(stream)),
+           "theta_residual_svd")
 
 
 def theta_linear_forward_noalloc(X, W0, s, U, V, Y, stream=None) -> None:

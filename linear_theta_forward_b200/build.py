@@ -23,7 +23,7 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libtheta.so")
 
 SOURCES = ["theta_api.cu", "stream_kernels.cu", "prelude_kernels.cu", "simt_kernels.cu", "umma_kernels.cu",
-           "gemv_kernels.cu", "noalloc.cu"]
+           "gemv_kernels.cu", "svd_kernels.cu", "noalloc.cu"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ARCH + [

@@ -60,6 +60,13 @@ bool launch_forward_gemv(const LaunchCtx& c, const void* X, const void* W0, cons
                          const void* V, int64_t M, int64_t O, int64_t I, int r, void* Y, void* ws,
                          cudaError_t* e);
 
+// ---- randomized SVD of a residual (svd_kernels.cu): R [O, I] in dt, omega
+// fp32 [samples, I]; U [O, rank], V [I, rank] in dt; ws of svd_workspace_bytes.
+int svd_max_samples();
+size_t svd_workspace_bytes(int64_t O, int64_t I, int samples, int rank);
+cudaError_t launch_residual_svd(const LaunchCtx& c, theta_dtype dt, const void* R, int64_t O, int64_t I, int rank,
+                                int samples, int power_iters, const float* omega, void* U, void* V, void* ws);
+
 // ---- tensor-core paths (umma_kernels.cu): bf16
 size_t forward_umma_workspace_bytes(int64_t M, int r);
 // Returns THETA_OK or a theta_status; CUDA errors are reported via *cuda_err.

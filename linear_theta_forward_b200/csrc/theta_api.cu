@@ -345,10 +345,29 @@ THETA_API int theta_linear_gate_up_forward(const void* X, int64_t M, int64_t I, 
   return st;
 }
 
+THETA_API int theta_residual_svd(const void* R, int64_t O, int64_t I, theta_dtype dt, int rank, int samples,
+                                 int power_iters, const float* omega, void* U, void* V, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (!valid_dt(dt)) return fail(THETA_ERR_INVALID_ARG, "theta_residual_svd: bad dtype %d", (int)dt);
+  if (O < 1 || I < 1 || rank < 1 || samples < rank || power_iters < 0 || power_iters > 8)
+    return fail(THETA_ERR_INVALID_ARG,
+                "theta_residual_svd: need O, I >= 1, 1 <= rank <= samples and 0 <= power_iters <= 8");
+  if (samples > svd_max_samples() || samples > O || samples > I)
+    return fail(THETA_ERR_UNSUPPORTED, "theta_residual_svd: samples must be <= min(%d, O, I)", svd_max_samples());
+  if (!R || !omega || !U || !V) return fail(THETA_ERR_INVALID_ARG, "theta_residual_svd: NULL pointer");
+  const size_t need = svd_workspace_bytes(O, I, samples, rank);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(THETA_ERR_WORKSPACE, "theta_residual_svd: need %zu bytes of 16-byte aligned workspace", need);
+  LaunchCtx c;
+  int st = make_ctx(stream, &c);
+  if (st) return st;
+  CHECK_LAUNCH(launch_residual_svd(c, dt, R, O, I, rank, samples, power_iters, omega, U, V, workspace),
+               "theta_residual_svd launch");
+  return THETA_OK;
+}
+
 THETA_API int theta_workspace_size(int op, int64_t M, int64_t O, int64_t I, int rank, theta_dtype dt,
                                    size_t* bytes) {
-  (void)O;
-  (void)I;
   if (!bytes) return fail(THETA_ERR_INVALID_ARG, "theta_workspace_size: bytes is NULL");
   if (!valid_dt(dt)) return fail(THETA_ERR_INVALID_ARG, "theta_workspace_size: bad dtype %d", (int)dt);
   switch (op) {
@@ -360,6 +379,11 @@ THETA_API int theta_workspace_size(int op, int64_t M, int64_t O, int64_t I, int 
     case THETA_OP_GATE_UP_FORWARD:
       if (M < 1 || rank < 0) return fail(THETA_ERR_INVALID_ARG, "theta_workspace_size: bad M or rank");
       *bytes = gate_up_umma_workspace_bytes(M, rank);
+      return THETA_OK;
+    case THETA_OP_RESIDUAL_SVD:  // M carries the number of samples
+      if (M < 1 || rank < 1 || M < rank || O < 1 || I < 1)
+        return fail(THETA_ERR_INVALID_ARG, "theta_workspace_size: bad samples, rank or sizes");
+      *bytes = svd_workspace_bytes(O, I, (int)M, rank);
       return THETA_OK;
   }
   return fail(THETA_ERR_INVALID_ARG, "theta_workspace_size: unknown op %d", op);

@@ -98,6 +98,20 @@ def test_validation_happens_before_any_cuda_call(lib):
                                             None) == -3                                          # I % 8 != 0
 
 
+def test_residual_svd_validation(lib):
+    raw = lib.lib
+    p = ctypes.c_void_p(16)
+    assert raw.theta_residual_svd(p, 64, 64, 0, 0, 8, 1, p, p, p, p, 1 << 30, None) == -1     # rank 0
+    assert raw.theta_residual_svd(p, 64, 64, 0, 9, 8, 1, p, p, p, p, 1 << 30, None) == -1     # rank > samples
+    assert raw.theta_residual_svd(p, 64, 64, 0, 4, 8, 9, p, p, p, p, 1 << 30, None) == -1     # power_iters > 8
+    assert raw.theta_residual_svd(p, 200, 200, 0, 4, 97, 1, p, p, p, p, 1 << 30, None) == -2  # samples > 96
+    assert raw.theta_residual_svd(p, 64, 20, 0, 4, 24, 1, p, p, p, p, 1 << 30, None) == -2    # samples > I
+    assert raw.theta_residual_svd(p, 64, 64, 0, 4, 8, 1, p, p, p, None, 0, None) == -6        # no workspace
+    small = lib.theta_workspace_size(lib.THETA_OP_RESIDUAL_SVD, 8, 64, 64, 4, lib.THETA_F32)
+    big = lib.theta_workspace_size(lib.THETA_OP_RESIDUAL_SVD, 74, 21504, 5376, 64, lib.THETA_BF16)
+    assert small >= 4 * (2 * 64 * 8 + 3 * 8 * 64) and big > small
+
+
 def test_gate_up_workspace_covers_both_projections(lib):
     for M, r in [(1, 8), (16, 32), (300, 64)]:
         one = lib.theta_workspace_size(lib.THETA_OP_LINEAR_FORWARD, M, 64, 64, r, lib.THETA_BF16)
