@@ -166,6 +166,87 @@ def randomized_svd(R, rank: int, omega, power_iters: int = 0):
     return (Q @ Ub[:, :rank]) * sig[:rank], Wt[:rank].T.copy()
 
 
+# ----------------------------------------------------------------- NVFP4
+# The pages name NVFP4 for weight bytes ("Quality" -- What NVFP4 quantization
+# costs; 3.18x smaller weights) without defining it. Published NVFP4: 4-bit
+# E2M1 elements, one FP8 E4M3 scale per 16 consecutive elements of a row,
+# and one FP32 scale per tensor. Every rounding decision below is taken in
+# fp32 with round-to-nearest-even, as the GPU takes it.
+F32 = np.float32
+
+
+def _grid_round(x, values):
+    """Round non-negative fp32 x to the nearest entry of `values` (ascending,
+    index = code), ties to the even code; above the top: the top (saturate)."""
+    x = np.asarray(x, dtype=F64)
+    v = np.asarray(values, dtype=F64)
+    hi = np.clip(np.searchsorted(v, x, side="left"), 1, len(v) - 1)
+    lo = hi - 1
+    dl, dh = x - v[lo], v[hi] - x
+    pick_hi = (dh < dl) | ((dh == dl) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo)
+    code = np.where(x >= v[-1], len(v) - 1, code)
+    return code.astype(np.int64)
+
+
+def e2m1_values() -> np.ndarray:
+    """Non-negative E2M1 magnitudes by code 0..7: 1 sign, 2 exponent (bias 1), 1 mantissa bit."""
+    return np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def e4m3_values() -> np.ndarray:
+    """Non-negative finite FP8 E4M3 values by code 0..126 (bias 7, 3 mantissa
+    bits, subnormals below 2^-6, largest 448; code 127 is NaN)."""
+    out = []
+    for c in range(127):
+        e, m = c >> 3, c & 7
+        out.append(m / 8.0 * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7))
+    return np.array(out)
+
+
+def nvfp4_quantize(W):
+    """W [O, I] (I a multiple of 16) -> (codes uint8 [O, I/2], element 2j in
+    the low nibble of byte j; scales uint8 [O, I/16], E4M3 codes; g fp32).
+
+    amax over the tensor; g = amax / (6 * 448); per block of 16: the block
+    scale b = blockmax / 6 relative to g, rounded to E4M3; the element scale
+    is E4M3(b) * g, and each element w * (1 / scale) is rounded to E2M1 with
+    its sign. A zero block (or tensor) gets zero codes.
+    """
+    w = np.asarray(W, dtype=F32)
+    O, I = w.shape
+    amax = F32(np.max(np.abs(w))) if w.size else F32(0)
+    g = F32(amax / F32(2688.0))
+    blk = np.abs(w).reshape(O, I // 16, 16).max(axis=2).astype(F32)
+    sb = (blk / F32(6.0)).astype(F32)
+    ratio = (sb / g).astype(F32) if g > 0 else np.zeros_like(sb)
+    sq = _grid_round(ratio, e4m3_values())
+    scale = (e4m3_values()[sq].astype(F32) * g).astype(F32)
+    inv = np.where(scale > 0, (F32(1.0) / np.where(scale > 0, scale, F32(1.0))).astype(F32), F32(0.0)).astype(F32)
+    x = (w.reshape(O, I // 16, 16) * inv[:, :, None]).astype(F32)
+    mag = _grid_round(np.abs(x), e2m1_values())
+    code = (mag | np.where((x < 0) & (mag > 0), 8, 0)).reshape(O, I).astype(np.uint8)
+    codes = (code[:, 0::2] | (code[:, 1::2] << 4)).astype(np.uint8)
+    return codes, sq.astype(np.uint8), g
+
+
+def nvfp4_dequantize(codes, scales, g) -> np.ndarray:
+    """The fp64 weights an NVFP4 encoding stands for: E2M1(code) * E4M3(scale) * g."""
+    c = np.asarray(codes, dtype=np.uint8)
+    O = c.shape[0]
+    el = np.empty((O, c.shape[1] * 2), dtype=np.int64)
+    el[:, 0::2], el[:, 1::2] = c & 15, c >> 4
+    mag = e2m1_values()[el & 7] * np.where(el & 8, -1.0, 1.0)
+    sc = e4m3_values()[np.asarray(scales, dtype=np.int64)]
+    return mag * np.repeat(sc, 16, axis=1) * F64(g)
+
+
+def linear_forward_nvfp4(X, codes, scales, g, s, U, V, out_dtype: str = "f64") -> np.ndarray:
+    """The theta forward with W0 given in NVFP4: the projection by the
+    dequantized shared block, s ⊙ (X·Ŵ0ᵀ) + (X·V)·Uᵀ."""
+    return linear_forward(X, nvfp4_dequantize(codes, scales, g), s, U, V, out_dtype)
+
+
 def reconstruct(s, W0, U, V, out_dtype: str = "f64") -> np.ndarray:
     """reconstruct_weight(s, W0, U, V) = diag(s)·W0 + U·Vᵀ
     ("The theta bundle" -- the approximation formula and Key layout)."""

@@ -315,7 +315,56 @@ def check_randomized_svd(o):
     assert U0.shape == (O, 0) and V0.shape == (I, 0)
 
 
-# --------------------------------------------------------------- pipeline# --------------------------------------------------------------- pipeline
+def check_nvfp4(o):
+    """NVFP4: the E2M1 and E4M3 grids, round-to-nearest-even with saturation
+    (E4M3 against torch's float8_e4m3fn cast), exact round trip for weights on
+    the grid, the error bound, zero blocks, packing order and the byte count."""
+    import torch
+    e2, e4 = o.e2m1_values(), o.e4m3_values()
+    assert list(e2) == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert len(e4) == 127 and e4[126] == 448.0 and e4[1] == 2.0 ** -9 and e4[56] == 1.0 and e4[8] == 2.0 ** -6
+    # E4M3 rounding of in-range values equals torch's cast (RNE), ties included
+    x = np.concatenate([np.linspace(0, 448, 20001), e4[1:] * (1 + 2.0 ** -4), (e4[1:] + e4[:-1]) / 2])
+    x = x[x <= 448].astype(np.float32)
+    codes = o._grid_round(x, e4) if hasattr(o, "_grid_round") else None
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert codes is not None and np.array_equal(e4[codes], ref)
+    # E2M1 ties go to the even code; above 6 saturates
+    xs = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0, 100.0, 0.26, 0.74], dtype=np.float32)
+    assert list(e2[o._grid_round(xs, e2)]) == [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0, 6.0, 6.0, 0.5, 0.5]
+    rng = _rng(31)
+    # weights on the grid come back exactly: every block holds its max 6*s*g
+    g = np.float32(2.0 ** -12)
+    O, I = 3, 64
+    sq = rng.integers(8, 127, size=(O, I // 16))
+    sq[0, 0] = 126  # the tensor max sets g
+    q = e2[rng.integers(0, 8, size=(O, I))] * rng.choice([-1.0, 1.0], size=(O, I))
+    q[:, ::16] = 6.0
+    W = (q * np.repeat(e4[sq], 16, axis=1) * g).astype(np.float32)
+    c, sc, gg = o.nvfp4_quantize(W)
+    assert gg == g and np.array_equal(sc, sq.astype(np.uint8))
+    assert np.array_equal(o.nvfp4_dequantize(c, sc, gg), W.astype(np.float64))
+    assert c.shape == (O, I // 2) and c.dtype == np.uint8
+    assert (c[0, 0] & 15) == 7 and (int(q[0, 1] < 0) << 3 | int(np.where(e2 == abs(q[0, 1]))[0][0])) == c[0, 0] >> 4
+    # random weights: each element within a quarter of its block's max
+    W = (rng.standard_normal((8, 128)) * 0.02).astype(np.float32)
+    W[2, 16:32] = 0.0
+    c, sc, gg = o.nvfp4_quantize(W)
+    D = o.nvfp4_dequantize(c, sc, gg)
+    bmax = np.repeat(np.abs(W).reshape(8, 8, 16).max(axis=2), 16, axis=1)
+    assert np.all(np.abs(D - W) <= 0.25 * bmax + 1e-30)
+    assert np.all(D[2, 16:32] == 0) and sc[2, 1] == 0
+    assert (c.nbytes + sc.nbytes) / W.size == 0.5625  # 3.56x fewer bytes than bf16
+    z, zs, zg = o.nvfp4_quantize(np.zeros((2, 32), np.float32))
+    assert zg == 0 and not z.any() and not zs.any()
+    # the forward with an NVFP4 shared block is the forward with its dequantized values
+    X = rng.standard_normal((3, 128))
+    s_, U, V = rng.standard_normal(8), rng.standard_normal((8, 4)), rng.standard_normal((128, 4))
+    assert np.allclose(o.linear_forward_nvfp4(X, c, sc, gg, s_, U, V), o.linear_forward(X, D, s_, U, V),
+                       rtol=1e-13, atol=1e-13)
+
+
+# --------------------------------------------------------------- pipeline# --------------------------------------------------------------- pipeline# --------------------------------------------------------------- pipeline
 def check_decompose(o):
     rng = _rng(9)
     L, O, I = 4, 6, 10
@@ -394,6 +443,6 @@ def check_gate_up(o):
     assert not np.allclose(Y, o.gate_up_forward(X, up, gate))
 
 
-ALL_CHECKS = [check_gelu, check_gate_up, check_randomized_svd, check_round, check_bands, check_band_mean, check_row_scale, check_residual,
+ALL_CHECKS = [check_gelu, check_gate_up, check_randomized_svd, check_nvfp4, check_round, check_bands, check_band_mean, check_row_scale, check_residual,
               check_reconstruct, check_frob, check_forward, check_svd, check_decompose,
               check_frob_statistics]

@@ -154,7 +154,28 @@ def _m_rsvd_sigma_in_v(R, rank, omega, power_iters=0):
     return U / np.where(n == 0, 1, n), V * n
 
 
+def _m_nvfp4_high_nibble_first(W):
+    c, sc, g = oracle.nvfp4_quantize(W)
+    return ((c >> 4) | (c << 4)).astype(np.uint8), sc, g
+
+
+def _m_nvfp4_ties_away(x, values):
+    v = np.asarray(values, np.float64)
+    x = np.asarray(x, np.float64)
+    hi = np.clip(np.searchsorted(v, x, side="left"), 1, len(v) - 1)
+    lo = hi - 1
+    code = np.where(v[hi] - x <= x - v[lo], hi, lo)
+    return np.where(x >= v[-1], len(v) - 1, code).astype(np.int64)
+
+
+def _m_nvfp4_no_global_scale(codes, scales, g):
+    return oracle.nvfp4_dequantize(codes, scales, 1.0)
+
+
 MUTANTS = {
+    "nvfp4_high_nibble_first": dict(nvfp4_quantize=_m_nvfp4_high_nibble_first),
+    "nvfp4_ties_away_from_zero": dict(_grid_round=_m_nvfp4_ties_away),
+    "nvfp4_drops_global_scale": dict(nvfp4_dequantize=_m_nvfp4_no_global_scale),
     "rsvd_sample_not_orthonormalized": dict(randomized_svd=_m_rsvd_unorthonormalized),
     "rsvd_sigma_in_v": dict(randomized_svd=_m_rsvd_sigma_in_v),
     "gelu_erf_form": dict(gelu_tanh=_m_gelu_erf),
