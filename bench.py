@@ -649,6 +649,33 @@ def run_op(args):
         # both weights streamed once, X read once, one output written
         nbytes = 2 * bytes_forward(M, O, I, r) - M * I * BF16 - M * O * BF16
         nflops = 2 * flops_forward(M, O, I, r)
+    elif args.op == "forward_nvfp4":
+        nbuf = args.bufs if args.b2b else 1
+        X = syn.device_normal((M, I), 1.0, seed, "X", M, I)
+        qws = torch.empty(16, dtype=torch.uint8, device="cuda")
+        probs = []
+        for k in range(nbuf):
+            W0 = syn.device_normal((O, I), 0.02, seed + k, "W0", O, I)
+            codes = torch.empty(O, I // 2, dtype=torch.uint8, device="cuda")
+            scales = torch.empty(O, I // 16, dtype=torch.uint8, device="cuda")
+            g = torch.empty(1, dtype=torch.float32, device="cuda")
+            theta.theta_nvfp4_quantize(W0, codes, scales, g, qws)
+            del W0
+            s = 1.0 + syn.device_normal((O,), 0.05, seed + k, "s", O, dtype="f32")
+            U = syn.device_normal((O, r), 0.01, seed + k, "U", O, r) if r else None
+            V = syn.device_normal((I, r), 0.01, seed + k, "V", I, r) if r else None
+            probs.append((codes, scales, g, s, U, V, torch.empty(M, O, dtype=torch.bfloat16, device="cuda")))
+        nb = theta.theta_workspace_size(theta.THETA_OP_LINEAR_FORWARD_NVFP4, M, O, I, r, theta.THETA_BF16)
+        ws = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
+        turn = [0]
+
+        def call():
+            codes, scales, g, s, U, V, Y = probs[turn[0] % nbuf]
+            turn[0] += 1
+            theta.theta_linear_forward_nvfp4(X, codes, scales, g, s, U, V, Y, ws)
+        # the NVFP4 block (0.5625 bytes per weight) instead of bf16 W0
+        nbytes = bytes_forward(M, O, I, r) - O * I * BF16 + O * I * 9 // 16
+        nflops = flops_forward(M, O, I, r)
     elif args.op == "svd":
         # randomized SVD of one residual: rank r, r + 10 samples, 2 subspace iterations
         k, q = min(r + 10, O, I), 2
@@ -702,7 +729,7 @@ def run_op(args):
         torch.cuda.synchronize()
         ms = a.elapsed_time(b) / args.iters
         l2 = "calls back to back, no flush (mean of %d)" % args.iters
-        if args.op in ("forward", "gate_up"):
+        if args.op in ("forward", "forward_nvfp4", "gate_up"):
             l2 += ", cycling over %d independent problems" % args.bufs
     else:
         times = []
@@ -742,7 +769,7 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-rows", type=int, default=32)
-    ap.add_argument("--op", choices=["forward", "gate_up", "reconstruct", "prelude", "frob", "svd"],
+    ap.add_argument("--op", choices=["forward", "forward_nvfp4", "gate_up", "reconstruct", "prelude", "frob", "svd"],
                     help="time one entry point on one problem instead of the whole step")
     ap.add_argument("--M", type=int, default=256)
     ap.add_argument("--O", type=int, default=21504)

@@ -65,7 +65,9 @@ typedef enum {
   THETA_OP_FROB_ERROR = 0,
   THETA_OP_LINEAR_FORWARD = 1,
   THETA_OP_GATE_UP_FORWARD = 2,
-  THETA_OP_RESIDUAL_SVD = 3
+  THETA_OP_RESIDUAL_SVD = 3,
+  THETA_OP_NVFP4_QUANTIZE = 4,
+  THETA_OP_LINEAR_FORWARD_NVFP4 = 5
 } theta_op;
 
 /* How the tensor-core kernels size their grids (see theta_set_policy). */
@@ -251,6 +253,44 @@ int theta_linear_gate_up_forward(const void* X, int64_t M, int64_t I, int64_t O,
                                  const void* V_gate, const void* W0_up, const float* s_up, const void* U_up,
                                  const void* V_up, void* Y, void* workspace, size_t workspace_bytes,
                                  void* stream);
+
+/*
+ * theta_nvfp4_quantize -- encodes a shared block W0 in NVFP4, the 4-bit
+ * weight format the pages measure ("Quality" -- What NVFP4 quantization
+ * costs: 3.18x smaller weights), at 0.5625 bytes per weight: E2M1 elements,
+ * one FP8 E4M3 scale per 16 consecutive elements of a row, one FP32 scale per
+ * tensor. Every decision in fp32, round-to-nearest-even, saturating:
+ *   g = amax|W0| / (6 * 448); per block: sq = E4M3(max|w| / 6 / g);
+ *   code = E2M1(w * (1 / (E4M3value(sq) * g))) with the sign of w (+0 for a
+ *   value that rounds to zero). The weight it stands for: E2M1 * E4M3 * g.
+ *
+ *   W0 [O, I] bf16 (I a multiple of 32, 16-byte aligned); codes uint8
+ *   [O, I/2] (element 2j in the low nibble of byte j; 16-byte aligned); scales
+ *   uint8 [O, I/16] (E4M3 codes; 2-byte aligned); g: device fp32 scalar,
+ *   written. workspace: 16 bytes (theta_workspace_size(THETA_OP_NVFP4_QUANTIZE)).
+ */
+int theta_nvfp4_quantize(const void* W0, int64_t O, int64_t I, void* codes, void* scales, float* g,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * theta_linear_forward_nvfp4 -- theta_linear_forward with the shared block
+ * given in NVFP4 (from theta_nvfp4_quantize): Y = s (.) (X . W0q^T) +
+ * (X . V) . U^T with W0q the dequantized block, for one or two tokens --
+ * the decode case, where the HBM bytes of W0 set the time and NVFP4 cuts
+ * them 3.56x. A CUDA-core sweep: X is first scaled per token by a power of
+ * two into fp16 (|x| <= 2^9, so no block sum can leave fp16's range); each
+ * pair of codes is widened to f16x2 by the Blackwell E2M1 conversion; a
+ * block's 16 products are summed by packed fp16 FMAs, scaled in fp32 by its
+ * E4M3 scale, and the row sum multiplied by g and the token's power of two.
+ *   X [M, I], U [O, rank], V [I, rank], Y [M, O] bf16; s fp32 [O]; codes,
+ *   scales, g as written by theta_nvfp4_quantize. M <= 2 (else
+ *   THETA_ERR_UNSUPPORTED); I a multiple of 32; O, rank multiples of 8.
+ *   workspace: theta_workspace_size(THETA_OP_LINEAR_FORWARD_NVFP4, M, O, I,
+ *   rank, THETA_BF16) bytes (T = X.V and X in fp16).
+ */
+int theta_linear_forward_nvfp4(const void* X, int64_t M, int64_t I, const void* codes, const void* scales,
+                               const float* g, int64_t O, const float* s, const void* U, const void* V, int rank,
+                               void* Y, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * theta_linear_forward_noalloc -- theta_linear_forward for callers that

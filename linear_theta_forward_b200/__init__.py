@@ -16,6 +16,7 @@ import numpy as np
 __all__ = [
     "ThetaError", "THETA_F32", "THETA_BF16", "THETA_OP_FROB_ERROR", "THETA_OP_LINEAR_FORWARD",
     "THETA_OP_GATE_UP_FORWARD", "theta_linear_gate_up_forward", "THETA_OP_RESIDUAL_SVD", "theta_residual_svd",
+    "THETA_OP_NVFP4_QUANTIZE", "THETA_OP_LINEAR_FORWARD_NVFP4", "theta_nvfp4_quantize", "theta_linear_forward_nvfp4",
     "THETA_MAX_LAYERS", "LIB_PATH", "lib",
     "theta_version", "theta_status_string", "theta_last_error", "theta_band_index",
     "theta_band_mean", "theta_row_scale", "theta_residual", "theta_decompose_prelude",
@@ -27,7 +28,8 @@ __all__ = [
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtheta.so")
 
 THETA_F32, THETA_BF16 = 0, 1
-THETA_OP_FROB_ERROR, THETA_OP_LINEAR_FORWARD, THETA_OP_GATE_UP_FORWARD, THETA_OP_RESIDUAL_SVD = 0, 1, 2, 3
+(THETA_OP_FROB_ERROR, THETA_OP_LINEAR_FORWARD, THETA_OP_GATE_UP_FORWARD, THETA_OP_RESIDUAL_SVD, THETA_OP_NVFP4_QUANTIZE,
+ THETA_OP_LINEAR_FORWARD_NVFP4) = 0, 1, 2, 3, 4, 5
 THETA_POLICY_LATENCY, THETA_POLICY_THROUGHPUT = 0, 1
 THETA_MAX_LAYERS = 256
 
@@ -53,6 +55,9 @@ _SIGNATURES = {
     "theta_frob_error": (_int, _vp, _vp, _i64, _int, _vp, _vp, _sz, _vp),
     "theta_linear_forward": (_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp, _sz, _vp),
     "theta_linear_forward_noalloc": (_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp),
+    "theta_nvfp4_quantize": (_int, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _sz, _vp),
+    "theta_linear_forward_nvfp4": (_int, _vp, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _int, _vp, _vp, _sz,
+                                   _vp),
     "theta_residual_svd": (_int, _vp, _i64, _i64, _int, _int, _int, _int, _vp, _vp, _vp, _vp, _sz, _vp),
     "theta_linear_gate_up_forward": (_int, _vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                      _vp, _vp, _sz, _vp),
@@ -254,6 +259,30 @@ def theta_linear_gate_up_forward(X, gate, up, Y, workspace=None, stream=None) ->
         _ptr(Ug, "U_gate", optional=True), _ptr(Vg, "V_gate", optional=True), _ptr(W0u, "W0_up"), _ptr(su, "s_up"),
         _ptr(Uu, "U_up", optional=True), _ptr(Vu, "V_up", optional=True), _ptr(Y, "Y"), ws_ptr, ws_bytes,
         _stream(stream)), "theta_linear_gate_up_forward")
+
+
+def theta_nvfp4_quantize(W0, codes, scales, g, workspace, stream=None) -> None:
+    """Encode W0 [O, I] bf16 in NVFP4: codes uint8 [O, I/2], scales uint8
+    [O, I/16] (E4M3), g fp32 device scalar [1]; workspace >= 16 bytes."""
+    O, I = W0.shape
+    _check(_load().theta_nvfp4_quantize(_ptr(W0, "W0"), O, I, _ptr(codes, "codes"), _ptr(scales, "scales"),
+                                        _ptr(g, "g"), _ptr(workspace, "workspace"),
+                                        workspace.numel() * workspace.element_size(), _stream(stream)),
+           "theta_nvfp4_quantize")
+
+
+def theta_linear_forward_nvfp4(X, codes, scales, g, s, U, V, Y, workspace=None, stream=None) -> None:
+    """Y [M, O] = s * (X W0q^T) + (X V) U^T with W0q the NVFP4 block (M <= 2)."""
+    M, I = X.shape
+    O = codes.shape[0]
+    rank = 0 if U is None else U.shape[1]
+    ws_ptr = _ptr(workspace, "workspace", optional=True)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_load().theta_linear_forward_nvfp4(_ptr(X, "X"), M, I, _ptr(codes, "codes"), _ptr(scales, "scales"),
+                                              _ptr(g, "g"), O, _ptr(s, "s"), _ptr(U, "U", optional=True),
+                                              _ptr(V, "V", optional=True), rank, _ptr(Y, "Y"), ws_ptr, ws_bytes,
+                                              _stream(stream)),
+           "theta_linear_forward_nvfp4")
 
 
 def theta_residual_svd(R, rank, omega, U, V, workspace, power_iters=2, stream=None) -> None:

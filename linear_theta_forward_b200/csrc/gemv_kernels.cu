@@ -21,6 +21,8 @@
 // the partial sums of T in a fixed order. The partial sums, U and s are
 // reached through pointers passed through after_wait(), so the compiler
 // cannot schedule their loads above the wait.
+#include <cuda_fp16.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -39,6 +41,7 @@ constexpr int64_t kMaxElements = (int64_t)32 << 20;
 constexpr int kMaxRank = 256;
 constexpr int kMaxRowsPerWarp = 64;
 constexpr int kUnroll = 4;  // 16-byte loads in flight per lane
+constexpr int kUnrollFp4 = 8;  // the same for NVFP4 codes (a row has 4x fewer)
 constexpr int kXvParts = 16;  // slices of I in the T = X.V partial sums
 
 struct GemvArgs {
@@ -47,6 +50,11 @@ struct GemvArgs {
   const float* s;
   const bf16* U;
   const float* t_parts;  // [kXvParts][M][r] partial sums of T = X.V
+  const uint8_t* codes;   // NVFP4 W0: E2M1 pairs [O, I/2], element 2j in the low nibble
+  const uint8_t* scales;  // NVFP4 W0: E4M3 block scales [O, I/16]
+  const float* g;         // NVFP4 W0: the tensor scale (device scalar)
+  const __half* x16;      // NVFP4: X / 2^e[m] in fp16 [M, I]
+  const float* xscale;    // NVFP4: 2^e[m]
   bf16* Y;
   int64_t O, I;
   int r;
@@ -127,6 +135,27 @@ __device__ __forceinline__ float sum_f32x2(uint64_t p) {
   return lo + hi;
 }
 
+// Two E2M1 codes (one byte, element 2j in the low nibble) -> two floats,
+// and two E4M3 codes (low byte first) -> two floats, by the Blackwell
+// conversions to f16x2; every E2M1 and E4M3 value is exact in fp16.
+// A word of 8 E2M1 codes (element 2j in the low nibble of byte j) as four
+// f16x2: h[q] holds elements 2q (low half) and 2q + 1.
+__device__ __forceinline__ void e2m1x8_to_h2(uint32_t w, uint32_t (&h)[4]) {
+  asm("{.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(w));
+}
+__device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t two_bytes) {
+  uint32_t h;
+  asm("{.reg .b16 u; cvt.u16.u32 u, %1; cvt.rn.f16x2.e4m3x2 %0, u;}" : "=r"(h) : "r"(two_bytes));
+  return __half22float2(*reinterpret_cast<__half2*>(&h));
+}
+
 // 8 bf16 -> 4 fp32 pairs (a bf16 is the high half of its fp32 value)
 __device__ __forceinline__ void bf16x8_to_f32x2(const uint4& v, uint64_t (&p)[4]) {
   const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -134,7 +163,7 @@ __device__ __forceinline__ void bf16x8_to_f32x2(const uint4& v, uint64_t (&p)[4]
   for (int q = 0; q < 4; ++q) p[q] = f32x2(__uint_as_float(w[q] << 16), __uint_as_float(w[q] & 0xffff0000u));
 }
 
-template <int M>
+template <int M, bool FP4>
 __global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_constant__ GemvArgs a) {
   __shared__ float dots[kWarps][kMaxRowsPerWarp][M];
   __shared__ float tsh[M][kMaxRank];
@@ -143,16 +172,111 @@ __global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_consta
   const bf16* W0 = a.W0;
   const float* s = a.s;
   const bf16* U = a.U;
+  const uint8_t* codes = a.codes;
+  const uint8_t* scales = a.scales;
+  const float* gp = a.g;
   if (!a.early) {
     pdl_wait();
-    after_wait(X), after_wait(W0), after_wait(s), after_wait(U);
+    after_wait(X), after_wait(W0), after_wait(s), after_wait(U), after_wait(codes), after_wait(scales), after_wait(gp);
   }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   const int64_t I = a.I, nv = I / 8;
   const int64_t row_lo = (int64_t)blockIdx.x * kWarps * a.rpw;
   const uint4* x = reinterpret_cast<const uint4*>(X);
-  for (int k = 0; k < a.rpw; ++k) {
+  if constexpr (FP4) {
+    // NVFP4 W0: a lane takes 16-byte chunks of codes (32 weights, two scale
+    // blocks) and the two scale bytes beside them. Two weights widen to an
+    // f16x2 in one conversion; X comes prescaled into fp16 (|x| <= 2^9, so a
+    // block's 16 products, each at most 6 * 2^9, sum far below fp16's
+    // limit); a block is summed by packed fp16 FMAs, each rounding once,
+    // then added in fp32 after its E4M3 scale.
+    //
+    // A row has only I/32 chunks, a few per lane, so the warp takes its rows
+    // kUnrollFp4 at a time and walks them group by group (a group: 32
+    // chunks, one per lane): the group's X is loaded once into registers
+    // and used for every row of the batch, and the batch's code loads are
+    // all in flight together. X is laid out so that a group's loads are
+    // contiguous across the warp (see nvfp4_x_prep_kernel).
+    const __half* x16 = a.x16;
+    const float* xsc = a.xscale;
+    after_wait(x16), after_wait(xsc);
+    const float gval = __ldg(gp);
+    float xs[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) xs[m] = __ldg(xsc + m) * gval;
+    const int nch = (int)(I / 32);  // chunks of a row
+    const int cj = (nch + 31) / 32;  // groups of a row
+    const uint4* xh = reinterpret_cast<const uint4*>(x16) + lane;
+    const int64_t first = row_lo + warp;
+    const int nrows = first < a.O ? (int)min((int64_t)a.rpw, ceil_div(a.O - first, kWarps)) : 0;
+    const int64_t cstep = (I / 32) * kWarps;  // uint4 of codes from one of the warp's rows to the next
+    const int64_t sstep = (I / 32) * kWarps;  // pairs of scale bytes, the same
+    for (int k0 = 0; k0 < nrows; k0 += kUnrollFp4) {
+      const uint4* cb = reinterpret_cast<const uint4*>(codes + (first + (int64_t)k0 * kWarps) * (I / 2)) + lane;
+      const unsigned short* sb =
+          reinterpret_cast<const unsigned short*>(scales + (first + (int64_t)k0 * kWarps) * (I / 16)) + lane;
+      float acc[kUnrollFp4][M];
+#pragma unroll
+      for (int u = 0; u < kUnrollFp4; ++u)
+#pragma unroll
+        for (int m = 0; m < M; ++m) acc[u][m] = 0.f;
+      for (int G = 0; G < cj; ++G) {
+        const bool vok = lane + 32 * G < nch;
+        uint4 cv[kUnrollFp4];
+        uint32_t sv[kUnrollFp4];
+#pragma unroll
+        for (int u = 0; u < kUnrollFp4; ++u) {
+          const bool ok = vok && k0 + u < nrows;
+          cv[u] = ok ? __ldcs(cb + u * cstep + 32 * G) : make_uint4(0, 0, 0, 0);
+          sv[u] = ok ? (uint32_t)__ldcs(sb + u * sstep + 32 * G) : 0u;
+        }
+        if (vok) {
+          uint4 xq[M][4];  // the group's 32 values of X for this lane's chunk
+#pragma unroll
+          for (int m = 0; m < M; ++m)
+#pragma unroll
+            for (int h = 0; h < 4; ++h) xq[m][h] = __ldg(xh + ((int64_t)m * cj + G) * 128 + 32 * h);
+#pragma unroll
+          for (int u = 0; u < kUnrollFp4; ++u) {
+            if (k0 + u >= nrows) break;
+            const float2 sc = e4m3x2_to_f32(sv[u]);
+            const uint32_t wd[4] = {cv[u].x, cv[u].y, cv[u].z, cv[u].w};
+#pragma unroll
+            for (int m = 0; m < M; ++m) {
+#pragma unroll
+              for (int b = 0; b < 2; ++b) {
+                __half2 p = __float2half2_rn(0.f);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  const uint32_t w32 = wd[2 * b + h];
+                  const uint4 xv = xq[m][2 * b + h];
+                  const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                  uint32_t wh[4];
+                  e2m1x8_to_h2(w32, wh);
+#pragma unroll
+                  for (int q = 0; q < 4; ++q)
+                    p = __hfma2(*reinterpret_cast<const __half2*>(&wh[q]), *reinterpret_cast<const __half2*>(&xw[q]), p);
+                }
+                const float2 pf = __half22float2(p);
+                acc[u][m] = fmaf(pf.x + pf.y, b == 0 ? sc.x : sc.y, acc[u][m]);
+              }
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnrollFp4; ++u) {
+        if (k0 + u >= nrows) break;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          const float d = warp_sum(acc[u][m]) * xs[m];
+          if (lane == 0) dots[warp][k0 + u][m] = d;
+        }
+      }
+    }
+  }
+  for (int k = 0; k < (FP4 ? 0 : a.rpw); ++k) {
     const int64_t o = row_lo + warp + (int64_t)k * kWarps;
     if (o >= a.O) break;
     const uint4* w = reinterpret_cast<const uint4*>(W0 + o * I);
@@ -223,19 +347,20 @@ __global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_consta
 }
 
 // CTAs of this kernel one SM holds at once (registers and threads decide).
-template <int M>
+template <int M, bool FP4>
 int resident_ctas(int device) {
   static int cached[64] = {};
   if (!cached[device]) {
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_rows_kernel<M>, kThreads, 0) != cudaSuccess || n < 1)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_rows_kernel<M, FP4>, kThreads, 0) != cudaSuccess ||
+        n < 1)
       n = 1;
     cached[device] = n;
   }
   return cached[device];
 }
 
-template <int M>
+template <int M, bool FP4 = false>
 cudaError_t launch_m(const LaunchCtx& c, GemvArgs a, const void* V) {
   if (a.r > 0) {
     cudaError_t e = launch_pdl(xv_parts_kernel<M>, dim3(kXvParts), dim3(kThreads), 0, c.stream, 1, a.X,
@@ -243,10 +368,10 @@ cudaError_t launch_m(const LaunchCtx& c, GemvArgs a, const void* V) {
     if (e != cudaSuccess) return e;
   }
   // the fewest rows per warp that keep every CTA resident in one wave
-  const int64_t capacity = (int64_t)c.num_sms * resident_ctas<M>(c.device) * kWarps;
+  const int64_t capacity = (int64_t)c.num_sms * resident_ctas<M, FP4>(c.device) * kWarps;
   a.rpw = (int)ceil_div(a.O, capacity);
   const int64_t grid = ceil_div(a.O, (int64_t)kWarps * a.rpw);
-  return launch_pdl(gemv_rows_kernel<M>, dim3((unsigned)grid), dim3(kThreads), 0, c.stream, 1, a);
+  return launch_pdl(gemv_rows_kernel<M, FP4>, dim3((unsigned)grid), dim3(kThreads), 0, c.stream, 1, a);
 }
 
 }  // namespace
@@ -277,6 +402,192 @@ bool launch_forward_gemv(const LaunchCtx& c, const void* X, const void* W0, cons
   a.r = r;
   a.early = r > 0 ? 1 : 0;
   *e = M == 1 ? launch_m<1>(c, a, V) : launch_m<2>(c, a, V);
+  return true;
+}
+
+}  // namespace theta
+
+namespace theta {
+
+namespace {
+
+// ------------------------------------------------------------ NVFP4 encode
+// max |w| over the tensor into *amax_bits (fp32 bits; for non-negative
+// floats the integer order is the float order, so atomicMax is exact and
+// the result independent of the order of the CTAs).
+__global__ void __launch_bounds__(256) nvfp4_amax_kernel(const bf16* __restrict__ W, int64_t nvec,
+                                                         unsigned* __restrict__ amax_bits) {
+  pdl_enter(W);
+  __shared__ float red[256 / 32];
+  float mx = 0.f;
+  const uint4* w4 = reinterpret_cast<const uint4*>(W);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t v = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v < nvec; v += stride) {
+    float f[8];
+    unpack(__ldcs(w4 + v), f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = mx;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float b = 0.f;
+    for (int i = 0; i < 256 / 32; ++i) b = fmaxf(b, red[i]);
+    atomicMax(amax_bits, __float_as_uint(b));
+  }
+}
+
+// One thread per block of 16 weights. Every decision in fp32 with
+// round-to-nearest-even: g = amax / (6 * 448); block scale
+// E4M3(blockmax / 6 / g) (saturating); element code E2M1(w * (1 / (E4M3 * g)))
+// (saturating, a negative value that rounds to zero is stored as +0).
+__global__ void __launch_bounds__(256) nvfp4_quant_kernel(const bf16* __restrict__ W, int64_t nblocks,
+                                                          const unsigned* __restrict__ amax_bits,
+                                                          uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                                                          float* __restrict__ g_out) {
+  pdl_enter(W, amax_bits);
+  const float g = __fdiv_rn(__uint_as_float(*amax_bits), 2688.0f);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *g_out = g;
+  const uint4* w4 = reinterpret_cast<const uint4*>(W);
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
+    float w[16];
+    unpack(w4[2 * b], *reinterpret_cast<float(*)[8]>(w));
+    unpack(w4[2 * b + 1], *reinterpret_cast<float(*)[8]>(w + 8));
+    float bmax = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) bmax = fmaxf(bmax, fabsf(w[e]));
+    const float ratio = g > 0.f ? __fdiv_rn(__fdiv_rn(bmax, 6.0f), g) : 0.f;
+    uint16_t sq16;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(sq16) : "f"(0.f), "f"(ratio));
+    const uint32_t sq = sq16 & 0xffu;
+    const float scale = __fmul_rn(e4m3x2_to_f32(sq).x, g);
+    const float inv = scale > 0.f ? __fdiv_rn(1.0f, scale) : 0.f;
+    uint32_t word[2] = {0u, 0u};
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      uint16_t byte;
+      asm("{.reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %1, %2; cvt.u16.u8 %0, t;}"
+          : "=h"(byte)
+          : "f"(__fmul_rn(w[2 * j + 1], inv)), "f"(__fmul_rn(w[2 * j], inv)));
+      uint32_t lo = byte & 15u, hi = (byte >> 4) & 15u;
+      if ((lo & 7u) == 0) lo = 0;  // -0 -> +0
+      if ((hi & 7u) == 0) hi = 0;
+      word[j / 4] |= (lo | (hi << 4)) << (8 * (j % 4));
+    }
+    reinterpret_cast<uint2*>(codes)[b] = make_uint2(word[0], word[1]);
+    scales[b] = (uint8_t)sq;
+  }
+}
+
+// X [M, I] bf16 -> X / 2^e in fp16 with 2^e >= max|x| / 2^9 (a power of
+// two, so the scaling is exact; with |x / 2^e| <= 2^9 a block's sum of 16
+// products with E2M1 weights, at most 6 each, stays below 2^16 * 0.75 and so
+// within fp16); one CTA per token.
+//
+// Layout: the sweep's lane l at step G reads chunk v = 32 G + l (32 values
+// of X) in four 16-byte loads h = 0..3; X[32 v + 8 h .. + 7] is stored at
+// 16-byte slot G * 128 + h * 32 + l of the token's ceil(I / 1024) * 128, so
+// each load of a step is one contiguous 512-byte run across the warp.
+__global__ void __launch_bounds__(256) nvfp4_x_prep_kernel(const bf16* __restrict__ X, int64_t I,
+                                                           __half* __restrict__ x16, float* __restrict__ xscale) {
+  pdl_enter(X);
+  __shared__ float red[256 / 32];
+  __shared__ float pw;
+  const int64_t m = blockIdx.x;
+  const uint4* xr = reinterpret_cast<const uint4*>(X + m * I);
+  const int64_t n8 = I / 8;
+  float mx = 0.f;
+  for (int64_t i = threadIdx.x; i < n8; i += blockDim.x) {
+    float f[8];
+    unpack(__ldg(xr + i), f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = mx;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float b = 0.f;
+    for (int k = 0; k < 256 / 32; ++k) b = fmaxf(b, red[k]);
+    int k = 0;
+    if (b > 0.f) frexpf(b, &k);  // b <= 2^k
+    const int e = max(-120, min(120, k - 9));  // 2^e >= b / 2^9, 1 / 2^e finite
+    pw = ldexpf(1.0f, e);
+    xscale[m] = pw;
+  }
+  __syncthreads();
+  const float inv = 1.0f / pw;  // a power of two: exact
+  uint4* dst = reinterpret_cast<uint4*>(x16) + m * ceil_div(I, 1024) * 128;
+  for (int64_t i = threadIdx.x; i < n8; i += blockDim.x) {
+    float f[8];
+    unpack(__ldg(xr + i), f);
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      __half2 h = __floats2half2_rn(f[2 * e] * inv, f[2 * e + 1] * inv);
+      w[e] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    const int64_t v = i / 4, h = i % 4;
+    dst[(v / 32) * 128 + h * 32 + v % 32] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_nvfp4_quantize(const LaunchCtx& c, const void* W, int64_t O, int64_t I, void* codes, void* scales,
+                                  float* g, void* ws) {
+  unsigned* amax = static_cast<unsigned*>(ws);
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned), c.stream);
+  if (e != cudaSuccess) return e;
+  const int64_t nvec = O * I / 8, nblocks = O * I / 16;
+  const auto grid = [&](int64_t n) {
+    int64_t b = ceil_div(n, 256);
+    return (unsigned)(b > 8 * (int64_t)c.num_sms ? 8 * (int64_t)c.num_sms : b < 1 ? 1 : b);
+  };
+  e = launch_pdl(nvfp4_amax_kernel, dim3(grid(nvec)), dim3(256), 0, c.stream, 1, static_cast<const bf16*>(W), nvec,
+                 amax);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(nvfp4_quant_kernel, dim3(grid(nblocks)), dim3(256), 0, c.stream, 1, static_cast<const bf16*>(W),
+                    nblocks, (const unsigned*)amax, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales), g);
+}
+
+size_t forward_nvfp4_workspace_bytes(int64_t M, int64_t I, int r) {
+  return (forward_gemv_workspace_bytes(M, r) + 255) / 256 * 256 + (size_t)(M * ceil_div(I, 1024) * 2048) + 256;
+}
+
+bool launch_forward_nvfp4(const LaunchCtx& c, const void* X, const void* codes, const void* scales, const float* g,
+                          const float* s, const void* U, const void* V, int64_t M, int64_t O, int64_t I, int r,
+                          void* Y, void* ws, cudaError_t* e) {
+  *e = cudaSuccess;
+  if (M < 1 || M > kMaxTokens || r > kMaxRank || I % 32) return false;
+  if (ceil_div(O, (int64_t)c.num_sms * kWarps) > kMaxRowsPerWarp) return false;
+  // workspace: T's partial sums, then X in fp16 and its per-token scales
+  const size_t tbytes = (forward_gemv_workspace_bytes(M, r) + 255) / 256 * 256;
+  __half* x16 = reinterpret_cast<__half*>(static_cast<uint8_t*>(ws) + tbytes);
+  float* xscale = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + tbytes + M * ceil_div(I, 1024) * 2048);
+  *e = launch_pdl(nvfp4_x_prep_kernel, dim3((unsigned)M), dim3(256), 0, c.stream, 1, static_cast<const bf16*>(X), I,
+                  x16, xscale);
+  if (*e != cudaSuccess) return true;
+  GemvArgs a = {};
+  a.X = static_cast<const bf16*>(X);
+  a.s = s;
+  a.U = static_cast<const bf16*>(U);
+  a.t_parts = static_cast<const float*>(ws);
+  a.x16 = x16;
+  a.xscale = xscale;
+  a.codes = static_cast<const uint8_t*>(codes);
+  a.scales = static_cast<const uint8_t*>(scales);
+  a.g = g;
+  a.Y = static_cast<bf16*>(Y);
+  a.O = O;
+  a.I = I;
+  a.r = r;
+  a.early = r > 0 ? 1 : 0;
+  *e = M == 1 ? launch_m<1, true>(c, a, V) : launch_m<2, true>(c, a, V);
   return true;
 }
 

@@ -60,6 +60,17 @@ bool launch_forward_gemv(const LaunchCtx& c, const void* X, const void* W0, cons
                          const void* V, int64_t M, int64_t O, int64_t I, int r, void* Y, void* ws,
                          cudaError_t* e);
 
+// ---- NVFP4 shared block (gemv_kernels.cu): encode W0 [O, I] bf16 into E2M1
+// codes [O, I/2], E4M3 block scales [O, I/16] and the tensor scale *g (ws: 4
+// bytes of scratch); the forward for one or two tokens from that encoding
+// (false: does not fit the sweep; ws of forward_nvfp4_workspace_bytes).
+cudaError_t launch_nvfp4_quantize(const LaunchCtx& c, const void* W, int64_t O, int64_t I, void* codes, void* scales,
+                                  float* g, void* ws);
+size_t forward_nvfp4_workspace_bytes(int64_t M, int64_t I, int r);
+bool launch_forward_nvfp4(const LaunchCtx& c, const void* X, const void* codes, const void* scales, const float* g,
+                          const float* s, const void* U, const void* V, int64_t M, int64_t O, int64_t I, int r,
+                          void* Y, void* ws, cudaError_t* e);
+
 // ---- randomized SVD of a residual (svd_kernels.cu): R [O, I] in dt, omega
 // fp32 [samples, I]; U [O, rank], V [I, rank] in dt; ws of svd_workspace_bytes.
 int svd_max_samples();

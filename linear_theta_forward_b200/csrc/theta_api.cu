@@ -366,6 +366,52 @@ THETA_API int theta_residual_svd(const void* R, int64_t O, int64_t I, theta_dtyp
   return THETA_OK;
 }
 
+THETA_API int theta_nvfp4_quantize(const void* W0, int64_t O, int64_t I, void* codes, void* scales, float* g,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  if (O < 1 || I < 1 || I % 32)
+    return fail(THETA_ERR_INVALID_ARG, "theta_nvfp4_quantize: need O >= 1 and I a positive multiple of 32");
+  if (!W0 || !codes || !scales || !g) return fail(THETA_ERR_INVALID_ARG, "theta_nvfp4_quantize: NULL pointer");
+  if (!aligned16(W0) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 1u) ||
+      (reinterpret_cast<uintptr_t>(g) & 3u))
+    return fail(THETA_ERR_ALIGNMENT, "theta_nvfp4_quantize: W0 and codes 16-byte, scales 2-byte, g 4-byte aligned");
+  if (!workspace || workspace_bytes < 16 || !aligned16(workspace))
+    return fail(THETA_ERR_WORKSPACE, "theta_nvfp4_quantize: need 16 bytes of 16-byte aligned workspace");
+  LaunchCtx c;
+  int st = make_ctx(stream, &c);
+  if (st) return st;
+  CHECK_LAUNCH(launch_nvfp4_quantize(c, W0, O, I, codes, scales, g, workspace), "theta_nvfp4_quantize launch");
+  return THETA_OK;
+}
+
+THETA_API int theta_linear_forward_nvfp4(const void* X, int64_t M, int64_t I, const void* codes, const void* scales,
+                                         const float* g, int64_t O, const float* s, const void* U, const void* V,
+                                         int rank, void* Y, void* workspace, size_t workspace_bytes, void* stream) {
+  if (M < 1 || I < 1 || O < 1 || rank < 0 || I % 32)
+    return fail(THETA_ERR_INVALID_ARG,
+                "theta_linear_forward_nvfp4: need M, O >= 1, rank >= 0 and I a positive multiple of 32");
+  if (!X || !codes || !scales || !g || !s || !Y || (rank > 0 && (!U || !V)))
+    return fail(THETA_ERR_INVALID_ARG, "theta_linear_forward_nvfp4: NULL pointer");
+  if (M > forward_gemv_max_tokens())
+    return fail(THETA_ERR_UNSUPPORTED, "theta_linear_forward_nvfp4: at most %d tokens (the decode sweep)",
+                forward_gemv_max_tokens());
+  if (!aligned16(X) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 1u) || !aligned16(Y) ||
+      (rank > 0 && (!aligned16(U) || !aligned16(V))) || O % 8 || rank % 8)
+    return fail(THETA_ERR_ALIGNMENT,
+                "theta_linear_forward_nvfp4: X, codes, Y, U, V 16-byte aligned, scales 2-byte; O, rank multiples of 8");
+  const size_t need = forward_nvfp4_workspace_bytes(M, I, rank);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(THETA_ERR_WORKSPACE, "theta_linear_forward_nvfp4: need %zu bytes of 16-byte aligned workspace",
+                need);
+  LaunchCtx c;
+  int st = make_ctx(stream, &c);
+  if (st) return st;
+  cudaError_t ce = cudaSuccess;
+  if (!launch_forward_nvfp4(c, X, codes, scales, g, s, U, V, M, O, I, rank, Y, workspace, &ce))
+    return fail(THETA_ERR_UNSUPPORTED, "theta_linear_forward_nvfp4: shape outside the decode sweep");
+  if (ce != cudaSuccess) return fail_cuda(ce, "theta_linear_forward_nvfp4 launch");
+  return THETA_OK;
+}
+
 THETA_API int theta_workspace_size(int op, int64_t M, int64_t O, int64_t I, int rank, theta_dtype dt,
                                    size_t* bytes) {
   if (!bytes) return fail(THETA_ERR_INVALID_ARG, "theta_workspace_size: bytes is NULL");
@@ -379,6 +425,13 @@ THETA_API int theta_workspace_size(int op, int64_t M, int64_t O, int64_t I, int 
     case THETA_OP_GATE_UP_FORWARD:
       if (M < 1 || rank < 0) return fail(THETA_ERR_INVALID_ARG, "theta_workspace_size: bad M or rank");
       *bytes = gate_up_umma_workspace_bytes(M, rank);
+      return THETA_OK;
+    case THETA_OP_NVFP4_QUANTIZE:
+      *bytes = 16;
+      return THETA_OK;
+    case THETA_OP_LINEAR_FORWARD_NVFP4:
+      if (M < 1 || rank < 0 || I < 1) return fail(THETA_ERR_INVALID_ARG, "theta_workspace_size: bad M, I or rank");
+      *bytes = forward_nvfp4_workspace_bytes(M, I, rank);
       return THETA_OK;
     case THETA_OP_RESIDUAL_SVD:  // M carries the number of samples
       if (M < 1 || rank < 1 || M < rank || O < 1 || I < 1)

@@ -98,6 +98,18 @@ def test_validation_happens_before_any_cuda_call(lib):
                                             None) == -3                                          # I % 8 != 0
 
 
+def test_nvfp4_validation(lib):
+    raw = lib.lib
+    p = ctypes.c_void_p(16)
+    assert raw.theta_nvfp4_quantize(p, 8, 48, p, p, p, p, 16, None) == -1        # I not a multiple of 32
+    assert raw.theta_nvfp4_quantize(p, 8, 64, p, p, p, None, 0, None) == -6      # no workspace
+    assert raw.theta_nvfp4_quantize(p, 8, 64, p, ctypes.c_void_p(17), p, p, 16, None) == -3  # odd scales
+    assert raw.theta_linear_forward_nvfp4(p, 4, 64, p, p, p, 8, p, p, p, 8, p, p, 1 << 20, None) == -2  # M > 2
+    assert raw.theta_linear_forward_nvfp4(p, 1, 64, p, p, p, 8, p, None, None, 8, p, p, 1 << 20, None) == -1
+    assert raw.theta_linear_forward_nvfp4(p, 1, 64, p, p, p, 8, p, p, p, 8, p, None, 0, None) == -6
+    assert lib.theta_workspace_size(lib.THETA_OP_NVFP4_QUANTIZE, 1, 8, 64, 0, lib.THETA_BF16) == 16
+
+
 def test_residual_svd_validation(lib):
     raw = lib.lib
     p = ctypes.c_void_p(16)
