@@ -277,16 +277,19 @@ int theta_nvfp4_quantize(const void* W0, int64_t O, int64_t I, void* codes, void
  * given in NVFP4 (from theta_nvfp4_quantize): Y = s (.) (X . W0q^T) +
  * (X . V) . U^T with W0q the dequantized block, for one or two tokens --
  * the decode case, where the HBM bytes of W0 set the time and NVFP4 cuts
- * them 3.56x. A CUDA-core sweep: X is first scaled per token by a power of
- * two into fp16 (|x| <= 2^9, so no block sum can leave fp16's range); each
- * pair of codes is widened to f16x2 by the Blackwell E2M1 conversion; a
- * block's 16 products are summed by packed fp16 FMAs, scaled in fp32 by its
- * E4M3 scale, and the row sum multiplied by g and the token's power of two.
+ * them 3.56x. A CUDA-core sweep: each CTA first writes X into shared
+ * memory in fp16, scaled by a power of two per group of 1024 values so that
+ * |x| <= 2^9 (no block sum can leave fp16's range); each pair of codes is
+ * widened to f16x2 by the Blackwell E2M1 conversion; a block's 16 products
+ * are summed by packed fp16 FMAs, scaled in fp32 by its E4M3 scale and the
+ * group's power of two, and the row sum multiplied by g.
  *   X [M, I], U [O, rank], V [I, rank], Y [M, O] bf16; s fp32 [O]; codes,
  *   scales, g as written by theta_nvfp4_quantize. M <= 2 (else
- *   THETA_ERR_UNSUPPORTED); I a multiple of 32; O, rank multiples of 8.
+ *   THETA_ERR_UNSUPPORTED); I a multiple of 32 and at most 49152 for one
+ *   token, 24576 for two (X must fit in shared memory; else
+ *   THETA_ERR_UNSUPPORTED); O, rank multiples of 8.
  *   workspace: theta_workspace_size(THETA_OP_LINEAR_FORWARD_NVFP4, M, O, I,
- *   rank, THETA_BF16) bytes (T = X.V and X in fp16).
+ *   rank, THETA_BF16) bytes (the partial sums of T = X.V; 0 at rank 0).
  */
 int theta_linear_forward_nvfp4(const void* X, int64_t M, int64_t I, const void* codes, const void* scales,
                                const float* g, int64_t O, const float* s, const void* U, const void* V, int rank,

@@ -23,6 +23,8 @@
 // cannot schedule their loads above the wait.
 #include <cuda_fp16.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -41,20 +43,22 @@ constexpr int64_t kMaxElements = (int64_t)32 << 20;
 constexpr int kMaxRank = 256;
 constexpr int kMaxRowsPerWarp = 64;
 constexpr int kUnroll = 4;  // 16-byte loads in flight per lane
-constexpr int kUnrollFp4 = 8;  // the same for NVFP4 codes (a row has 4x fewer)
+constexpr int kUnrollFp4 = 4;  // NVFP4: rows a warp takes at a time, one 16-byte load each
 constexpr int kXvParts = 16;  // slices of I in the T = X.V partial sums
+// With NVFP4 the sweep is 3.56x shorter, so T = X.V must finish sooner:
+// more, smaller slices.
+constexpr int kXvPartsFp4 = 64;
 
 struct GemvArgs {
   const bf16* X;
   const bf16* W0;
   const float* s;
   const bf16* U;
-  const float* t_parts;  // [kXvParts][M][r] partial sums of T = X.V
+  const float* t_parts;  // [nparts][M][r] partial sums of T = X.V
   const uint8_t* codes;   // NVFP4 W0: E2M1 pairs [O, I/2], element 2j in the low nibble
   const uint8_t* scales;  // NVFP4 W0: E4M3 block scales [O, I/16]
   const float* g;         // NVFP4 W0: the tensor scale (device scalar)
-  const __half* x16;      // NVFP4: X / 2^e[m] in fp16 [M, I]
-  const float* xscale;    // NVFP4: 2^e[m]
+  int nparts;             // slices of I in the T = X.V partial sums
   bf16* Y;
   int64_t O, I;
   int r;
@@ -73,7 +77,7 @@ xv_parts_kernel(const bf16* __restrict__ X, const bf16* __restrict__ V, int64_t 
   __shared__ float red[kThreads * 8 * M];  // [slice][m][column]
   pdl_enter(X, V);
   const int p = blockIdx.x;
-  const int64_t i0 = (int64_t)p * I / kXvParts, i1 = (int64_t)(p + 1) * I / kXvParts;
+  const int64_t i0 = (int64_t)p * I / gridDim.x, i1 = (int64_t)(p + 1) * I / gridDim.x;
   const int groups = r / 8;  // 16-byte column groups per row of V
   const int nslices = kThreads / groups;
   const int t = threadIdx.x, cg = t % groups, slice = t / groups;
@@ -187,31 +191,59 @@ __global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_consta
   if constexpr (FP4) {
     // NVFP4 W0: a lane takes 16-byte chunks of codes (32 weights, two scale
     // blocks) and the two scale bytes beside them. Two weights widen to an
-    // f16x2 in one conversion; X comes prescaled into fp16 (|x| <= 2^9, so a
-    // block's 16 products, each at most 6 * 2^9, sum far below fp16's
-    // limit); a block is summed by packed fp16 FMAs, each rounding once,
-    // then added in fp32 after its E4M3 scale.
+    // f16x2 in one conversion and meet X in fp16, scaled by a power of two
+    // per group of 1024 values so that |x| <= 2^9 (a block's 16 products, at
+    // most 6 * 2^9 each, then sum far below fp16's limit); a block is summed
+    // by packed fp16 FMAs, each rounding once, and added in fp32 after its
+    // E4M3 scale and the group's power of two.
     //
-    // A row has only I/32 chunks, a few per lane, so the warp takes its rows
-    // kUnrollFp4 at a time and walks them group by group (a group: 32
-    // chunks, one per lane): the group's X is loaded once into registers
-    // and used for every row of the batch, and the batch's code loads are
-    // all in flight together. X is laid out so that a group's loads are
-    // contiguous across the warp (see nvfp4_x_prep_kernel).
-    const __half* x16 = a.x16;
-    const float* xsc = a.xscale;
-    after_wait(x16), after_wait(xsc);
-    const float gval = __ldg(gp);
-    float xs[M];
-#pragma unroll
-    for (int m = 0; m < M; ++m) xs[m] = __ldg(xsc + m) * gval;
+    // First the CTA writes X so converted into shared memory: each warp
+    // takes groups (32 chunks, one per lane), reduces the group's largest
+    // |x| and stores lane l's 32 values at 16-byte slots
+    // group * 128 + h * 32 + l, h = 0..3 (conflict-free on both sides).
+    // Then a row has only I/32 chunks, a few per lane, so the warp takes its
+    // rows kUnrollFp4 at a time and walks them group by group: the group's X
+    // comes from shared memory once for every row of the batch, and the
+    // batch's code loads are all in flight together.
+    extern __shared__ uint4 xsm[];  // [M][cj][128] fp16 X, then float gsc[M][cj]
     const int nch = (int)(I / 32);  // chunks of a row
     const int cj = (nch + 31) / 32;  // groups of a row
-    const uint4* xh = reinterpret_cast<const uint4*>(x16) + lane;
+    float* gsc = reinterpret_cast<float*>(xsm + (size_t)M * cj * 128);
+    for (int it = warp; it < M * cj; it += kWarps) {
+      const int m = it / cj, v = 32 * (it - m * cj) + lane;
+      float f[4][8];
+      float mx = 0.f;
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const uint4 raw = v < nch ? __ldg(x + (int64_t)m * nv + 4 * v + h) : make_uint4(0, 0, 0, 0);
+        unpack(raw, f[h]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[h][e]));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      int k = 0;
+      if (mx > 0.f) frexpf(mx, &k);  // mx <= 2^k
+      const int e = max(-120, min(120, k - 9));  // 2^e >= mx / 2^9, both 2^e and 2^-e finite
+      const float inv = ldexpf(1.0f, -e);  // exact scaling
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          __half2 hv = __floats2half2_rn(f[h][2 * q] * inv, f[h][2 * q + 1] * inv);
+          w[q] = *reinterpret_cast<uint32_t*>(&hv);
+        }
+        xsm[it * 128 + 32 * h + lane] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      if (lane == 0) gsc[it] = ldexpf(1.0f, e);
+    }
+    __syncthreads();
+
+    const float gval = __ldg(gp);
     const int64_t first = row_lo + warp;
     const int nrows = first < a.O ? (int)min((int64_t)a.rpw, ceil_div(a.O - first, kWarps)) : 0;
-    const int64_t cstep = (I / 32) * kWarps;  // uint4 of codes from one of the warp's rows to the next
-    const int64_t sstep = (I / 32) * kWarps;  // pairs of scale bytes, the same
+    const int64_t cstep = (int64_t)nch * kWarps;  // chunks from one of the warp's rows to the next
     for (int k0 = 0; k0 < nrows; k0 += kUnrollFp4) {
       const uint4* cb = reinterpret_cast<const uint4*>(codes + (first + (int64_t)k0 * kWarps) * (I / 2)) + lane;
       const unsigned short* sb =
@@ -229,14 +261,17 @@ __global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_consta
         for (int u = 0; u < kUnrollFp4; ++u) {
           const bool ok = vok && k0 + u < nrows;
           cv[u] = ok ? __ldcs(cb + u * cstep + 32 * G) : make_uint4(0, 0, 0, 0);
-          sv[u] = ok ? (uint32_t)__ldcs(sb + u * sstep + 32 * G) : 0u;
+          sv[u] = ok ? (uint32_t)__ldcs(sb + u * cstep + 32 * G) : 0u;
         }
         if (vok) {
-          uint4 xq[M][4];  // the group's 32 values of X for this lane's chunk
+          uint4 xq[M][4];  // this lane's 32 values of X in the group
+          float gs[M];
 #pragma unroll
-          for (int m = 0; m < M; ++m)
+          for (int m = 0; m < M; ++m) {
 #pragma unroll
-            for (int h = 0; h < 4; ++h) xq[m][h] = __ldg(xh + ((int64_t)m * cj + G) * 128 + 32 * h);
+            for (int h = 0; h < 4; ++h) xq[m][h] = xsm[(m * cj + G) * 128 + 32 * h + lane];
+            gs[m] = gsc[m * cj + G];
+          }
 #pragma unroll
           for (int u = 0; u < kUnrollFp4; ++u) {
             if (k0 + u >= nrows) break;
@@ -249,17 +284,16 @@ __global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_consta
                 __half2 p = __float2half2_rn(0.f);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                  const uint32_t w32 = wd[2 * b + h];
                   const uint4 xv = xq[m][2 * b + h];
                   const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
                   uint32_t wh[4];
-                  e2m1x8_to_h2(w32, wh);
+                  e2m1x8_to_h2(wd[2 * b + h], wh);
 #pragma unroll
                   for (int q = 0; q < 4; ++q)
                     p = __hfma2(*reinterpret_cast<const __half2*>(&wh[q]), *reinterpret_cast<const __half2*>(&xw[q]), p);
                 }
                 const float2 pf = __half22float2(p);
-                acc[u][m] = fmaf(pf.x + pf.y, b == 0 ? sc.x : sc.y, acc[u][m]);
+                acc[u][m] = fmaf(pf.x + pf.y, (b == 0 ? sc.x : sc.y) * gs[m], acc[u][m]);
               }
             }
           }
@@ -270,7 +304,7 @@ __global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_consta
         if (k0 + u >= nrows) break;
 #pragma unroll
         for (int m = 0; m < M; ++m) {
-          const float d = warp_sum(acc[u][m]) * xs[m];
+          const float d = warp_sum(acc[u][m]) * gval;
           if (lane == 0) dots[warp][k0 + u][m] = d;
         }
       }
@@ -319,7 +353,7 @@ __global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_consta
   const int r = a.r;
   for (int i = threadIdx.x; i < M * r; i += kThreads) {
     float t = 0.f;
-    for (int p = 0; p < kXvParts; ++p) t += parts[(int64_t)p * M * r + i];
+    for (int p = 0; p < a.nparts; ++p) t += parts[(int64_t)p * M * r + i];
     tsh[i / r][i % r] = t;
   }
   __syncthreads();
@@ -346,16 +380,33 @@ __global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_consta
   }
 }
 
-// CTAs of this kernel one SM holds at once (registers and threads decide).
+// Dynamic shared memory of the NVFP4 sweep: X in fp16 and its group scales.
+constexpr size_t kFp4SmemMax = 200 << 10;
+size_t fp4_smem_bytes(int64_t M, int64_t I) {
+  const int64_t groups = M * ceil_div(I / 32, 32);
+  return (size_t)groups * 2048 + (size_t)ceil_div(groups * 4, 16) * 16;
+}
+
+// CTAs of this kernel one SM holds at once with `smem` bytes of dynamic
+// shared memory (registers, threads and shared memory decide).
 template <int M, bool FP4>
-int resident_ctas(int device) {
+int resident_ctas(int device, size_t smem) {
   static int cached[64] = {};
-  if (!cached[device]) {
+  static size_t cached_smem[64] = {};
+  if (!cached[device] || cached_smem[device] != smem) {
+    if (FP4) {
+      static bool opted[64] = {};
+      if (!opted[device]) {
+        cudaFuncSetAttribute(gemv_rows_kernel<M, FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kFp4SmemMax);
+        opted[device] = true;
+      }
+    }
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_rows_kernel<M, FP4>, kThreads, 0) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_rows_kernel<M, FP4>, kThreads, smem) != cudaSuccess ||
         n < 1)
       n = 1;
     cached[device] = n;
+    cached_smem[device] = smem;
   }
   return cached[device];
 }
@@ -363,15 +414,16 @@ int resident_ctas(int device) {
 template <int M, bool FP4 = false>
 cudaError_t launch_m(const LaunchCtx& c, GemvArgs a, const void* V) {
   if (a.r > 0) {
-    cudaError_t e = launch_pdl(xv_parts_kernel<M>, dim3(kXvParts), dim3(kThreads), 0, c.stream, 1, a.X,
+    cudaError_t e = launch_pdl(xv_parts_kernel<M>, dim3((unsigned)a.nparts), dim3(kThreads), 0, c.stream, 1, a.X,
                                static_cast<const bf16*>(V), a.I, a.r, const_cast<float*>(a.t_parts));
     if (e != cudaSuccess) return e;
   }
+  const size_t smem = FP4 ? fp4_smem_bytes(M, a.I) : 0;
   // the fewest rows per warp that keep every CTA resident in one wave
-  const int64_t capacity = (int64_t)c.num_sms * resident_ctas<M, FP4>(c.device) * kWarps;
+  const int64_t capacity = (int64_t)c.num_sms * resident_ctas<M, FP4>(c.device, smem) * kWarps;
   a.rpw = (int)ceil_div(a.O, capacity);
   const int64_t grid = ceil_div(a.O, (int64_t)kWarps * a.rpw);
-  return launch_pdl(gemv_rows_kernel<M, FP4>, dim3((unsigned)grid), dim3(kThreads), 0, c.stream, 1, a);
+  return launch_pdl(gemv_rows_kernel<M, FP4>, dim3((unsigned)grid), dim3(kThreads), smem, c.stream, 1, a);
 }
 
 }  // namespace
@@ -396,6 +448,7 @@ bool launch_forward_gemv(const LaunchCtx& c, const void* X, const void* W0, cons
   a.s = s;
   a.U = static_cast<const bf16*>(U);
   a.t_parts = static_cast<const float*>(ws);
+  a.nparts = kXvParts;
   a.Y = static_cast<bf16*>(Y);
   a.O = O;
   a.I = I;
@@ -482,60 +535,6 @@ __global__ void __launch_bounds__(256) nvfp4_quant_kernel(const bf16* __restrict
   }
 }
 
-// X [M, I] bf16 -> X / 2^e in fp16 with 2^e >= max|x| / 2^9 (a power of
-// two, so the scaling is exact; with |x / 2^e| <= 2^9 a block's sum of 16
-// products with E2M1 weights, at most 6 each, stays below 2^16 * 0.75 and so
-// within fp16); one CTA per token.
-//
-// Layout: the sweep's lane l at step G reads chunk v = 32 G + l (32 values
-// of X) in four 16-byte loads h = 0..3; X[32 v + 8 h .. + 7] is stored at
-// 16-byte slot G * 128 + h * 32 + l of the token's ceil(I / 1024) * 128, so
-// each load of a step is one contiguous 512-byte run across the warp.
-__global__ void __launch_bounds__(256) nvfp4_x_prep_kernel(const bf16* __restrict__ X, int64_t I,
-                                                           __half* __restrict__ x16, float* __restrict__ xscale) {
-  pdl_enter(X);
-  __shared__ float red[256 / 32];
-  __shared__ float pw;
-  const int64_t m = blockIdx.x;
-  const uint4* xr = reinterpret_cast<const uint4*>(X + m * I);
-  const int64_t n8 = I / 8;
-  float mx = 0.f;
-  for (int64_t i = threadIdx.x; i < n8; i += blockDim.x) {
-    float f[8];
-    unpack(__ldg(xr + i), f);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) mx = fmaxf(mx, fabsf(f[e]));
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x / 32] = mx;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    float b = 0.f;
-    for (int k = 0; k < 256 / 32; ++k) b = fmaxf(b, red[k]);
-    int k = 0;
-    if (b > 0.f) frexpf(b, &k);  // b <= 2^k
-    const int e = max(-120, min(120, k - 9));  // 2^e >= b / 2^9, 1 / 2^e finite
-    pw = ldexpf(1.0f, e);
-    xscale[m] = pw;
-  }
-  __syncthreads();
-  const float inv = 1.0f / pw;  // a power of two: exact
-  uint4* dst = reinterpret_cast<uint4*>(x16) + m * ceil_div(I, 1024) * 128;
-  for (int64_t i = threadIdx.x; i < n8; i += blockDim.x) {
-    float f[8];
-    unpack(__ldg(xr + i), f);
-    uint32_t w[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      __half2 h = __floats2half2_rn(f[2 * e] * inv, f[2 * e + 1] * inv);
-      w[e] = *reinterpret_cast<uint32_t*>(&h);
-    }
-    const int64_t v = i / 4, h = i % 4;
-    dst[(v / 32) * 128 + h * 32 + v % 32] = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-}
-
 }  // namespace
 
 cudaError_t launch_nvfp4_quantize(const LaunchCtx& c, const void* W, int64_t O, int64_t I, void* codes, void* scales,
@@ -556,29 +555,23 @@ cudaError_t launch_nvfp4_quantize(const LaunchCtx& c, const void* W, int64_t O, 
 }
 
 size_t forward_nvfp4_workspace_bytes(int64_t M, int64_t I, int r) {
-  return (forward_gemv_workspace_bytes(M, r) + 255) / 256 * 256 + (size_t)(M * ceil_div(I, 1024) * 2048) + 256;
+  (void)I;
+  return (M >= 1 && M <= kMaxTokens && r > 0) ? (size_t)kXvPartsFp4 * M * r * sizeof(float) : 0;
 }
 
 bool launch_forward_nvfp4(const LaunchCtx& c, const void* X, const void* codes, const void* scales, const float* g,
                           const float* s, const void* U, const void* V, int64_t M, int64_t O, int64_t I, int r,
                           void* Y, void* ws, cudaError_t* e) {
   *e = cudaSuccess;
-  if (M < 1 || M > kMaxTokens || r > kMaxRank || I % 32) return false;
+  if (M < 1 || M > kMaxTokens || r > kMaxRank || I % 32 || fp4_smem_bytes(M, I) > kFp4SmemMax) return false;
   if (ceil_div(O, (int64_t)c.num_sms * kWarps) > kMaxRowsPerWarp) return false;
-  // workspace: T's partial sums, then X in fp16 and its per-token scales
-  const size_t tbytes = (forward_gemv_workspace_bytes(M, r) + 255) / 256 * 256;
-  __half* x16 = reinterpret_cast<__half*>(static_cast<uint8_t*>(ws) + tbytes);
-  float* xscale = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + tbytes + M * ceil_div(I, 1024) * 2048);
-  *e = launch_pdl(nvfp4_x_prep_kernel, dim3((unsigned)M), dim3(256), 0, c.stream, 1, static_cast<const bf16*>(X), I,
-                  x16, xscale);
-  if (*e != cudaSuccess) return true;
+  if ((reinterpret_cast<uintptr_t>(X) & 15u) != 0) return false;
   GemvArgs a = {};
   a.X = static_cast<const bf16*>(X);
   a.s = s;
   a.U = static_cast<const bf16*>(U);
   a.t_parts = static_cast<const float*>(ws);
-  a.x16 = x16;
-  a.xscale = xscale;
+  a.nparts = (int)std::min<int64_t>(kXvPartsFp4, I);
   a.codes = static_cast<const uint8_t*>(codes);
   a.scales = static_cast<const uint8_t*>(scales);
   a.g = g;

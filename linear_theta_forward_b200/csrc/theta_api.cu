@@ -399,7 +399,7 @@ THETA_API int theta_linear_forward_nvfp4(const void* X, int64_t M, int64_t I, co
     return fail(THETA_ERR_ALIGNMENT,
                 "theta_linear_forward_nvfp4: X, codes, Y, U, V 16-byte aligned, scales 2-byte; O, rank multiples of 8");
   const size_t need = forward_nvfp4_workspace_bytes(M, I, rank);
-  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+  if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
     return fail(THETA_ERR_WORKSPACE, "theta_linear_forward_nvfp4: need %zu bytes of 16-byte aligned workspace",
                 need);
   LaunchCtx c;
