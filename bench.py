@@ -97,8 +97,10 @@ def prelude_launches(L, G, I, b=BF16, num_sms=148):
     return G + 1
 
 
-def step_accounting(model=MODEL, r=RANK, m_values=M_VALUES, g_values=G_VALUES):
-    """Per-stage algorithmic bytes / flops / kernel launches of one step."""
+def step_accounting(model=MODEL, r=RANK, m_values=M_VALUES, g_values=G_VALUES, grouped=True):
+    """Per-stage algorithmic bytes / flops / kernel launches of one step.
+    With `grouped`, a stage of one or two tokens is one grouped call (T = X.V
+    slices, their sums, one sweep: 3 launches, 1 at rank 0)."""
     L = model.num_layers
     stages = []
     for G in g_values:
@@ -117,8 +119,9 @@ def step_accounting(model=MODEL, r=RANK, m_values=M_VALUES, g_values=G_VALUES):
         stages.append(dict(name=f"reconstruct_G{G}", kind="reconstruct", bytes=rec, flops=0, launches=nf * L))
         stages.append(dict(name=f"frob_G{G}", kind="frob", bytes=fro, flops=0, launches=nf * L * 2))
         for m in m_values:
+            launches = (3 if r > 0 else 1) if grouped and m <= 2 else nf * L * (2 if r > 0 else 1)
             stages.append(dict(name=f"forward_m{m}_G{G}", kind=f"forward_m{m}", bytes=fwd[m][0],
-                               flops=fwd[m][1], launches=nf * L * (2 if r > 0 else 1)))
+                               flops=fwd[m][1], launches=launches))
     return stages
 
 
@@ -218,7 +221,7 @@ def result_line(*, value, unit, n_gpus, steps, warmup, ms_per_step, extra):
 class Workload:
     """All device tensors of one step, and the stage call lists."""
 
-    def __init__(self, theta, torch, seed=0, model=MODEL, r=RANK, streams=1):
+    def __init__(self, theta, torch, seed=0, model=MODEL, r=RANK, streams=1, grouped=True):
         self.theta, self.torch = theta, torch
         # independent calls of a stage (layers, families) spread round-robin
         # over this many streams; each stream has its own workspaces
@@ -248,6 +251,18 @@ class Workload:
                  for m in M_VALUES for (O, I) in model.shapes.values())
         self.fwd_ws = [torch.empty(max(wb, 256), dtype=torch.uint8, device=dev) for _ in range(streams)]
         self.bands = {G: theta.theta_band_index(L, G)[0] for G in G_VALUES}
+        # one or two tokens: every family of every layer in one grouped call
+        self.groups = {}
+        if grouped:
+            for G in G_VALUES:
+                for m in M_VALUES:
+                    if m <= 2:
+                        band = self.bands[G]
+                        self.groups[(G, m)] = theta.ForwardGroup([
+                            (self.X[(m, I)], self.W0[fam][band[l]], self.s[fam][l], self.U[fam][l], self.V[fam][l],
+                             self.Y[(m, fam, l)]) for fam, (O, I) in model.shapes.items() for l in range(L)])
+        gb = max([g.workspace_size() for g in self.groups.values()] + [256])
+        self.grp_ws = torch.empty(gb, dtype=torch.uint8, device=dev)
 
     # stage bodies ------------------------------------------------------
     def _fan_out(self, calls):
@@ -292,6 +307,9 @@ class Workload:
 
     def forward(self, G, m):
         t = self.theta
+        if (G, m) in self.groups:
+            t.theta_linear_forward_grouped(self.groups[(G, m)], self.grp_ws)
+            return
         band = self.bands[G]
         self._fan_out([lambda k, fam=fam, I=I, l=l: t.theta_linear_forward(
             self.X[(m, I)], self.W0[fam][band[l]], self.s[fam][l], self.U[fam][l], self.V[fam][l],
@@ -320,10 +338,24 @@ class Workload:
         return [self.frob_out] + list(self.Y.values()) + [s for fam in self.model.shapes for s in self.s[fam]]
 
 
-def kernel_source_hash():
+# The sources that define each stage's kernels and their launch code (the
+# shared device helpers included): a recorded ncu traffic figure stands only
+# while these files hash to the value recorded beside it.
+KIND_SOURCES = {
+    "prelude": ["prelude_kernels.cu", "stream_kernels.cu", "common.cuh", "umma_ptx.cuh"],
+    "reconstruct": ["umma_kernels.cu", "umma_ptx.cuh", "common.cuh"],
+    "frob": ["stream_kernels.cu", "common.cuh"],
+    "forward_m1": ["gemv_kernels.cu", "common.cuh"],
+    "forward_m16": ["umma_kernels.cu", "umma_ptx.cuh", "common.cuh"],
+    "forward_m256": ["umma_kernels.cu", "umma_ptx.cuh", "common.cuh"],
+}
+
+
+def kernel_source_hash(kind=None):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "linear_theta_forward_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    names = KIND_SOURCES.get(kind) or sorted(os.listdir(csrc))
+    for name in sorted(names):
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -331,14 +363,14 @@ def kernel_source_hash():
 
 def recorded_traffic(kind):
     """DRAM bytes per launch of a stage's main kernel from a committed ncu
-    capture, or None when the kernels changed since it was taken."""
+    capture, or None when that stage's kernel sources changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f)
     entry = rec.get(kind)
-    if not entry or entry.get("source_hash") != kernel_source_hash():
+    if not entry or entry.get("source_hash") != kernel_source_hash(kind):
         return None
     return entry.get("dram_bytes_per_launch")
 
@@ -448,8 +480,8 @@ def run_gpu(args):
     # many independent calls in flight at once: no split-K
     policy = theta.THETA_POLICY_THROUGHPUT if args.streams > 1 else theta.THETA_POLICY_LATENCY
     theta.theta_set_policy(policy)
-    wl = Workload(theta, torch, seed=rank, streams=args.streams)
-    stages = step_accounting()
+    wl = Workload(theta, torch, seed=rank, streams=args.streams, grouped=not args.per_call_decode)
+    stages = step_accounting(grouped=not args.per_call_decode)
     fns = wl.stage_fns()
     assert len(fns) == len(stages)
     stream = torch.cuda.Stream()
@@ -549,6 +581,7 @@ def run_gpu(args):
                                           "parallelism": f"independent replicas x{world}",
                                           "graphs": not args.no_graph, "streams": args.streams,
                                           "policy": "throughput" if policy else "latency",
+                                          "decode": "per call" if args.per_call_decode else "grouped",
                                           "l2": "inputs larger than L2 (>10 GB touched per step); no flush"},
                                "parts": parts,
                                "roofline": roofline,
@@ -676,6 +709,32 @@ def run_op(args):
         # the NVFP4 block (0.5625 bytes per weight) instead of bf16 W0
         nbytes = bytes_forward(M, O, I, r) - O * I * BF16 + O * I * 9 // 16
         nflops = flops_forward(M, O, I, r)
+    elif args.op == "grouped":
+        # every family of --layers Gemma-3-1B-shaped layers in one grouped call
+        # (or, with --per-call-decode, one theta_linear_forward per problem)
+        xs = {I_: syn.device_normal((M, I_), 1.0, seed, "X", M, I_) for (_, I_) in MODEL.shapes.values()}
+        probs = []
+        for fam, (O_, I_) in MODEL.shapes.items():
+            for l in range(L):
+                probs.append((xs[I_], syn.device_normal((O_, I_), 0.02, seed + l, "W0", fam),
+                              1.0 + syn.device_normal((O_,), 0.05, seed + l, "s", fam, dtype="f32"),
+                              syn.device_normal((O_, r), 0.01, seed + l, "U", fam) if r else None,
+                              syn.device_normal((I_, r), 0.01, seed + l, "V", fam) if r else None,
+                              torch.empty(M, O_, dtype=torch.bfloat16, device="cuda")))
+        if args.per_call_decode:
+            nb = max(theta.theta_workspace_size(theta.THETA_OP_LINEAR_FORWARD, M, O_, I_, r, theta.THETA_BF16)
+                     for (O_, I_) in MODEL.shapes.values())
+            ws = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
+
+            def call():
+                for X_, W0, s, U, V, Y in probs:
+                    theta.theta_linear_forward(X_, W0, s, U, V, Y, ws)
+        else:
+            group = theta.ForwardGroup(probs)
+            ws = torch.empty(max(group.workspace_size(), 256), dtype=torch.uint8, device="cuda")
+            call = lambda: theta.theta_linear_forward_grouped(group, ws)  # noqa: E731
+        nbytes = sum(bytes_forward(M, p[1].shape[0], p[1].shape[1], r) for p in probs)
+        nflops = sum(flops_forward(M, p[1].shape[0], p[1].shape[1], r) for p in probs)
     elif args.op == "svd":
         # randomized SVD of one residual: rank r, r + 10 samples, 2 subspace iterations
         k, q = min(r + 10, O, I), 2
@@ -764,12 +823,15 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
     ap.add_argument("--streams", type=int, default=16, help="streams the independent calls of a stage spread over")
+    ap.add_argument("--per-call-decode", action="store_true",
+                    help="one theta_linear_forward per problem for one or two tokens instead of a grouped call")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--skip-cpu", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-rows", type=int, default=32)
-    ap.add_argument("--op", choices=["forward", "forward_nvfp4", "gate_up", "reconstruct", "prelude", "frob", "svd"],
+    ap.add_argument("--op", choices=["forward", "forward_nvfp4", "gate_up", "grouped", "reconstruct", "prelude", "frob",
+                                     "svd"],
                     help="time one entry point on one problem instead of the whole step")
     ap.add_argument("--M", type=int, default=256)
     ap.add_argument("--O", type=int, default=21504)

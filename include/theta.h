@@ -48,6 +48,7 @@ extern "C" {
 
 #define THETA_VERSION 1
 #define THETA_MAX_LAYERS 256 /* layers per call of the band/prelude entry points */
+#define THETA_MAX_GROUP 256  /* problems per call of theta_linear_forward_grouped */
 
 typedef enum {
   THETA_OK = 0,
@@ -67,7 +68,8 @@ typedef enum {
   THETA_OP_GATE_UP_FORWARD = 2,
   THETA_OP_RESIDUAL_SVD = 3,
   THETA_OP_NVFP4_QUANTIZE = 4,
-  THETA_OP_LINEAR_FORWARD_NVFP4 = 5
+  THETA_OP_LINEAR_FORWARD_NVFP4 = 5,
+  THETA_OP_LINEAR_FORWARD_GROUPED = 6
 } theta_op;
 
 /* How the tensor-core kernels size their grids (see theta_set_policy). */
@@ -271,6 +273,47 @@ int theta_linear_gate_up_forward(const void* X, int64_t M, int64_t I, int64_t O,
  */
 int theta_nvfp4_quantize(const void* W0, int64_t O, int64_t I, void* codes, void* scales, float* g,
                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One problem of theta_linear_forward_grouped: the arguments of one bf16
+ * theta_linear_forward call (the token count M is shared by the group).
+ * 72 bytes, natural alignment; the field order is the ABI.
+ */
+typedef struct theta_forward_problem {
+  const void* X;   /* [M, I] bf16 */
+  const void* W0;  /* [O, I] bf16 */
+  const float* s;  /* [O] fp32 */
+  const void* U;   /* [O, rank] bf16; NULL when rank == 0 */
+  const void* V;   /* [I, rank] bf16; NULL when rank == 0 */
+  void* Y;         /* [M, O] bf16, written */
+  int64_t O;
+  int64_t I;
+  int64_t rank;
+} theta_forward_problem;
+
+/*
+ * theta_linear_forward_grouped -- `count` independent bf16 theta forwards of
+ * the same one or two tokens count, in one call ("The theta bundle" --
+ * approximation formula, applied to every projection of every layer: the
+ * decode step of a whole model, whose per-call latency dominates at small
+ * sizes). Each Y is what theta_linear_forward would write, up to fp32
+ * summation order. Three launches for the whole group: T = X.V of every
+ * problem (8 slices of I each), their fixed-order sums, and one CUDA-core
+ * sweep over the rows of all problems laid end to end.
+ *   problems         host array of `count` descriptors (read during the call
+ *                    only: sizes, validation)
+ *   problems_device  device copy of the same array (the kernels read it);
+ *                    the caller keeps it alive and unchanged until the work
+ *                    has run. The two must hold the same contents.
+ *   1 <= count <= THETA_MAX_GROUP; 1 <= M <= 2 (else THETA_ERR_UNSUPPORTED).
+ *   Per problem: O, I >= 1, 0 <= rank <= 256; I, O, rank multiples of 8 and
+ *   X, W0, s, U, V 16-byte aligned (else THETA_ERR_ALIGNMENT).
+ *   workspace: theta_workspace_size(THETA_OP_LINEAR_FORWARD_GROUPED, M,
+ *   count, 0, max rank over the problems, THETA_BF16) bytes (0 when every
+ *   rank is 0).
+ */
+int theta_linear_forward_grouped(const theta_forward_problem* problems, const theta_forward_problem* problems_device,
+                                 int count, int64_t M, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * theta_linear_forward_nvfp4 -- theta_linear_forward with the shared block

@@ -17,7 +17,8 @@ __all__ = [
     "ThetaError", "THETA_F32", "THETA_BF16", "THETA_OP_FROB_ERROR", "THETA_OP_LINEAR_FORWARD",
     "THETA_OP_GATE_UP_FORWARD", "theta_linear_gate_up_forward", "THETA_OP_RESIDUAL_SVD", "theta_residual_svd",
     "THETA_OP_NVFP4_QUANTIZE", "THETA_OP_LINEAR_FORWARD_NVFP4", "theta_nvfp4_quantize", "theta_linear_forward_nvfp4",
-    "THETA_MAX_LAYERS", "LIB_PATH", "lib",
+    "THETA_MAX_LAYERS", "LIB_PATH", "lib", "THETA_OP_LINEAR_FORWARD_GROUPED", "THETA_MAX_GROUP",
+    "theta_forward_problem", "ForwardGroup", "theta_linear_forward_grouped",
     "theta_version", "theta_status_string", "theta_last_error", "theta_band_index",
     "theta_band_mean", "theta_row_scale", "theta_residual", "theta_decompose_prelude",
     "theta_reconstruct", "theta_frob_error", "theta_linear_forward", "theta_workspace_size",
@@ -29,9 +30,10 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtheta.so
 
 THETA_F32, THETA_BF16 = 0, 1
 (THETA_OP_FROB_ERROR, THETA_OP_LINEAR_FORWARD, THETA_OP_GATE_UP_FORWARD, THETA_OP_RESIDUAL_SVD, THETA_OP_NVFP4_QUANTIZE,
- THETA_OP_LINEAR_FORWARD_NVFP4) = 0, 1, 2, 3, 4, 5
+ THETA_OP_LINEAR_FORWARD_NVFP4, THETA_OP_LINEAR_FORWARD_GROUPED) = 0, 1, 2, 3, 4, 5, 6
 THETA_POLICY_LATENCY, THETA_POLICY_THROUGHPUT = 0, 1
 THETA_MAX_LAYERS = 256
+THETA_MAX_GROUP = 256
 
 _i32p = ctypes.POINTER(ctypes.c_int32)
 _vp = ctypes.c_void_p
@@ -61,6 +63,7 @@ _SIGNATURES = {
     "theta_residual_svd": (_int, _vp, _i64, _i64, _int, _int, _int, _int, _vp, _vp, _vp, _vp, _sz, _vp),
     "theta_linear_gate_up_forward": (_int, _vp, _i64, _i64, _i64, _int, _int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                      _vp, _vp, _sz, _vp),
+    "theta_linear_forward_grouped": (_int, _vp, _vp, _int, _i64, _vp, _sz, _vp),
     "theta_workspace_size": (_int, _int, _i64, _i64, _i64, _int, _int, ctypes.POINTER(_sz)),
     "theta_device_status": (_int, _vp),
 }
@@ -241,6 +244,52 @@ def theta_linear_forward(X, W0, s, U, V, Y, workspace=None, stream=None) -> None
                                     _ptr(U, "U", optional=True), _ptr(V, "V", optional=True), rank,
                                     _dtype_code(X), _ptr(Y, "Y"), ws_ptr, ws_bytes, _stream(stream)),
            "theta_linear_forward")
+
+
+class theta_forward_problem(ctypes.Structure):
+    """One problem of theta_linear_forward_grouped (the C struct, 72 bytes)."""
+    _fields_ = [("X", _vp), ("W0", _vp), ("s", _vp), ("U", _vp), ("V", _vp), ("Y", _vp), ("O", _i64), ("I", _i64),
+                ("rank", _i64)]
+
+
+class ForwardGroup:
+    """The problem table of a grouped forward: `problems` is a list of
+    (X, W0, s, U, V, Y) tuples (U = V = None at rank 0) with one token count
+    M. Holds the host array, its device copy and references to the tensors,
+    so build it once and reuse it while the tensors stay where they are."""
+
+    def __init__(self, problems):
+        if not problems:
+            raise ValueError("ForwardGroup: no problems")
+        n = len(problems)
+        self.count = n
+        self.M = int(problems[0][0].shape[0])
+        self.rmax = 0
+        self.host = (theta_forward_problem * n)()
+        for i, (X, W0, s, U, V, Y) in enumerate(problems):
+            O, I = W0.shape
+            rank = 0 if U is None else int(U.shape[1])
+            self.rmax = max(self.rmax, rank)
+            self.host[i] = theta_forward_problem(_ptr(X, "X"), _ptr(W0, "W0"), _ptr(s, "s"),
+                                                 _ptr(U, "U", optional=True), _ptr(V, "V", optional=True),
+                                                 _ptr(Y, "Y"), O, I, rank)
+        raw = ctypes.string_at(ctypes.addressof(self.host), ctypes.sizeof(self.host))
+        import torch
+        self.device = torch.frombuffer(bytearray(raw), dtype=torch.uint8).to(problems[0][0].device)
+        self._tensors = problems
+
+    def workspace_size(self) -> int:
+        return theta_workspace_size(THETA_OP_LINEAR_FORWARD_GROUPED, self.M, self.count, 0, self.rmax, THETA_BF16)
+
+
+def theta_linear_forward_grouped(group: ForwardGroup, workspace=None, stream=None) -> None:
+    """Every problem's Y [M, O] = s * (X W0^T) + (X V) U^T in one call.
+    workspace: CUDA tensor of at least group.workspace_size() bytes (None if 0)."""
+    ws_ptr = _ptr(workspace, "workspace", optional=True)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_load().theta_linear_forward_grouped(ctypes.cast(group.host, _vp), _ptr(group.device, "problems_device"),
+                                                group.count, group.M, ws_ptr, ws_bytes, _stream(stream)),
+           "theta_linear_forward_grouped")
 
 
 def theta_linear_gate_up_forward(X, gate, up, Y, workspace=None, stream=None) -> None:

@@ -21,6 +21,12 @@
 // the partial sums of T in a fixed order. The partial sums, U and s are
 // reached through pointers passed through after_wait(), so the compiler
 // cannot schedule their loads above the wait.
+//
+// The same sweep also reads the shared block in NVFP4 (codes, E4M3 block
+// scales, fp32 tensor scale; the format the pages weigh in "Quality" -- what
+// NVFP4 quantization costs): 0.5625 bytes per weight instead of 2. Its rows are split evenly over one full wave of CTAs, each
+// warp taking a contiguous range; see the FP4 branch of gemv_rows_kernel.
+// The encoder (nvfp4_amax_kernel, nvfp4_quant_kernel) sits at the end.
 #include <cuda_fp16.h>
 
 #include <algorithm>
@@ -66,18 +72,15 @@ struct GemvArgs {
   int rpw;    // rows per warp; a CTA owns 8 * rpw consecutive rows
 };
 
-// parts[p][m][j] = sum over i in slice p of I of X[m, i] V[i, j]. A thread
-// owns 8 consecutive columns of V (one 16-byte load per row of V) and every
-// nslices-th row of the slice, four rows in flight; the row slices are then
-// combined in a fixed order. r is a multiple of 8 and at most 256.
+// out[m * r + j] = sum over i in [i0, i1) of X[m, i] V[i, j], by one CTA. A
+// thread owns 8 consecutive columns of V (one 16-byte load per row of V) and
+// every nslices-th row of the range, four rows in flight; the row slices are
+// then combined in a fixed order through shared memory. r is a multiple of 8
+// and at most 256.
 template <int M>
-__global__ void __launch_bounds__(kThreads)
-xv_parts_kernel(const bf16* __restrict__ X, const bf16* __restrict__ V, int64_t I, int r, float* __restrict__ parts) {
+__device__ __forceinline__ void xv_slice(const bf16* __restrict__ X, const bf16* __restrict__ V, int64_t I, int r,
+                                         int64_t i0, int64_t i1, float* red, float* __restrict__ out) {
   constexpr int kRowsInFlight = 4;
-  __shared__ float red[kThreads * 8 * M];  // [slice][m][column]
-  pdl_enter(X, V);
-  const int p = blockIdx.x;
-  const int64_t i0 = (int64_t)p * I / gridDim.x, i1 = (int64_t)(p + 1) * I / gridDim.x;
   const int groups = r / 8;  // 16-byte column groups per row of V
   const int nslices = kThreads / groups;
   const int t = threadIdx.x, cg = t % groups, slice = t / groups;
@@ -118,8 +121,19 @@ xv_parts_kernel(const bf16* __restrict__ X, const bf16* __restrict__ V, int64_t 
   for (int q = t; q < M * r; q += kThreads) {
     float sum = 0.f;
     for (int sl = 0; sl < nslices; ++sl) sum += red[sl * M * r + q];
-    parts[(int64_t)p * M * r + q] = sum;  // q = m * r + j
+    out[q] = sum;  // q = m * r + j
   }
+}
+
+// parts[p][m][j]: the sum over slice p (of gridDim.x) of I.
+template <int M>
+__global__ void __launch_bounds__(kThreads)
+xv_parts_kernel(const bf16* __restrict__ X, const bf16* __restrict__ V, int64_t I, int r, float* __restrict__ parts) {
+  __shared__ float red[kThreads * 8 * M];  // [slice][m][column]
+  pdl_enter(X, V);
+  const int p = blockIdx.x;
+  const int64_t i0 = (int64_t)p * I / gridDim.x, i1 = (int64_t)(p + 1) * I / gridDim.x;
+  xv_slice<M>(X, V, I, r, i0, i1, red, parts + (int64_t)p * M * r);
 }
 
 // Packed fp32 pairs (Blackwell fma.rn.f32x2: two fp32 FMAs per instruction).
@@ -188,6 +202,20 @@ __global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_consta
   const int64_t I = a.I, nv = I / 8;
   const int64_t row_lo = (int64_t)blockIdx.x * kWarps * a.rpw;
   const uint4* x = reinterpret_cast<const uint4*>(X);
+  // The rows this warp owns: o = rbase + k * rstride for k < nr.
+  int64_t rbase, rstride;
+  int nr;
+  if constexpr (FP4) {
+    // one wave of CTAs; each warp a contiguous, balanced range of rows
+    const int64_t nw = (int64_t)gridDim.x * kWarps, gw = (int64_t)blockIdx.x * kWarps + warp;
+    rbase = gw * a.O / nw;
+    rstride = 1;
+    nr = (int)((gw + 1) * a.O / nw - rbase);
+  } else {
+    rbase = row_lo + warp;
+    rstride = kWarps;
+    nr = rbase < a.O ? (int)min((int64_t)a.rpw, ceil_div(a.O - rbase, kWarps)) : 0;
+  }
   if constexpr (FP4) {
     // NVFP4 W0: a lane takes 16-byte chunks of codes (32 weights, two scale
     // blocks) and the two scale bytes beside them. Two weights widen to an
@@ -241,13 +269,13 @@ __global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_consta
     __syncthreads();
 
     const float gval = __ldg(gp);
-    const int64_t first = row_lo + warp;
-    const int nrows = first < a.O ? (int)min((int64_t)a.rpw, ceil_div(a.O - first, kWarps)) : 0;
-    const int64_t cstep = (int64_t)nch * kWarps;  // chunks from one of the warp's rows to the next
+    const int64_t first = rbase;
+    const int nrows = nr;
+    const int64_t cstep = (int64_t)nch * rstride;  // chunks from one of the warp's rows to the next
     for (int k0 = 0; k0 < nrows; k0 += kUnrollFp4) {
-      const uint4* cb = reinterpret_cast<const uint4*>(codes + (first + (int64_t)k0 * kWarps) * (I / 2)) + lane;
+      const uint4* cb = reinterpret_cast<const uint4*>(codes + (first + (int64_t)k0 * rstride) * (I / 2)) + lane;
       const unsigned short* sb =
-          reinterpret_cast<const unsigned short*>(scales + (first + (int64_t)k0 * kWarps) * (I / 16)) + lane;
+          reinterpret_cast<const unsigned short*>(scales + (first + (int64_t)k0 * rstride) * (I / 16)) + lane;
       float acc[kUnrollFp4][M];
 #pragma unroll
       for (int u = 0; u < kUnrollFp4; ++u)
@@ -357,9 +385,8 @@ __global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_consta
     tsh[i / r][i % r] = t;
   }
   __syncthreads();
-  for (int k = 0; k < a.rpw; ++k) {
-    const int64_t o = row_lo + warp + (int64_t)k * kWarps;
-    if (o >= a.O) break;
+  for (int k = 0; k < nr; ++k) {
+    const int64_t o = rbase + (int64_t)k * rstride;
     float rk[M];
 #pragma unroll
     for (int m = 0; m < M; ++m) rk[m] = 0.f;
@@ -377,6 +404,170 @@ __global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_consta
         if (m == lane) y = fmaf(__ldg(s + o), dots[warp][k][m], rk[m]);
       a.Y[(int64_t)lane * a.O + o] = __float2bfloat16_rn(y);
     }
+  }
+}
+
+// ------------------------------------------------------- grouped decode
+// Many independent forwards of one or two tokens in one call (every family
+// of every layer, say): three launches instead of two per problem. T = X.V
+// for all problems first (kGroupParts slices of I each, then a fixed-order
+// sum), then one sweep over the rows of all problems laid end to end, split
+// over one wave of CTAs by weight elements (equal bytes per warp, whatever
+// the row widths); a warp owns a contiguous range of those rows and takes
+// them kGroupRows at a time (dot products, rank terms, Y).
+constexpr int kGroupParts = 8;
+constexpr int kGroupRows = 4;    // rows of one problem a warp takes at a time
+constexpr int kGroupUnroll = 2;  // 16-byte loads per row in flight per lane
+constexpr int kMaxGroup = THETA_MAX_GROUP;
+
+struct GroupArgs {
+  const theta_forward_problem* P;  // device copy of the problem table
+  const float* T;                   // [count][M][rmax]: T = X.V, entry m * r + j
+  int64_t elems[kMaxGroup + 1];     // first weight element of each problem (rows end to end)
+  int32_t prefix[kMaxGroup + 1];    // first row of each problem; prefix[count] = all rows
+  int count;
+  int rmax;
+};
+static_assert(sizeof(GroupArgs) <= 4096, "kernel parameter space");
+
+// The first row (in the rows of all problems end to end) that starts at or
+// after weight element e: rows split at element boundaries, so warps given
+// equal element ranges stream equal bytes whatever each problem's width.
+__device__ __forceinline__ int64_t group_row_at(const GroupArgs& g, int64_t e) {
+  if (e >= g.elems[g.count]) return g.prefix[g.count];
+  int p = 0;  // the last problem with elems[p] <= e
+  for (int lo = 0, hi = g.count - 1; lo < hi;) {
+    const int mid = (lo + hi + 1) / 2;
+    if (g.elems[mid] <= e) lo = mid; else hi = mid - 1;
+    p = lo;
+  }
+  const int64_t rows = g.prefix[p + 1] - g.prefix[p];
+  const int64_t width = (g.elems[p + 1] - g.elems[p]) / rows;
+  return g.prefix[p] + min(rows, ceil_div(e - g.elems[p], width));
+}
+
+template <int M>
+__global__ void __launch_bounds__(kThreads)
+grouped_xv_kernel(const theta_forward_problem* __restrict__ P, int rmax, float* __restrict__ parts) {
+  __shared__ float red[kThreads * 8 * M];
+  pdl_enter(P);
+  const theta_forward_problem d = P[blockIdx.y];
+  const int r = (int)d.rank;
+  if (r == 0) return;
+  const int p = blockIdx.x;
+  const int64_t i0 = (int64_t)p * d.I / kGroupParts, i1 = (int64_t)(p + 1) * d.I / kGroupParts;
+  xv_slice<M>(static_cast<const bf16*>(d.X), static_cast<const bf16*>(d.V), d.I, r, i0, i1, red,
+              parts + ((int64_t)blockIdx.y * kGroupParts + p) * M * rmax);
+}
+
+template <int M>
+__global__ void __launch_bounds__(kThreads)
+grouped_t_kernel(const theta_forward_problem* __restrict__ P, int rmax, const float* __restrict__ parts,
+                 float* __restrict__ T) {
+  pdl_enter(P, parts);
+  const int b = blockIdx.x;
+  const int r = (int)P[b].rank;
+  for (int q = threadIdx.x; q < M * r; q += kThreads) {
+    float t = 0.f;
+    for (int p = 0; p < kGroupParts; ++p) t += parts[((int64_t)b * kGroupParts + p) * M * rmax + q];
+    T[(int64_t)b * M * rmax + q] = t;
+  }
+}
+
+template <int M>
+__global__ void __launch_bounds__(kThreads) grouped_rows_kernel(const __grid_constant__ GroupArgs g) {
+  const theta_forward_problem* P = g.P;
+  const float* T = g.T;
+  pdl_enter(P, T);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int64_t total = g.elems[g.count];
+  const int64_t nw = (int64_t)gridDim.x * kWarps, gw = (int64_t)blockIdx.x * kWarps + warp;
+  const int64_t r0 = group_row_at(g, gw * total / nw), r1 = group_row_at(g, (gw + 1) * total / nw);
+  if (r0 >= r1) return;
+  int p = 0;  // the problem holding row r0: the last p with prefix[p] <= r0
+  for (int lo = 0, hi = g.count - 1; lo < hi;) {
+    const int mid = (lo + hi + 1) / 2;
+    if (g.prefix[mid] <= r0) lo = mid; else hi = mid - 1;
+    p = lo;
+  }
+  theta_forward_problem d = P[p];
+  // batches of up to kGroupRows consecutive rows of one problem: their W0
+  // chunks are in flight together and share each load of X
+  for (int64_t row = r0; row < r1;) {
+    if (row >= g.prefix[p + 1]) {
+      while (row >= g.prefix[p + 1]) ++p;
+      d = P[p];
+    }
+    const int64_t o0 = row - g.prefix[p], I = d.I, nv = I / 8;
+    const int nb = (int)min((int64_t)kGroupRows, min(r1, (int64_t)g.prefix[p + 1]) - row);
+    const uint4* w = reinterpret_cast<const uint4*>(static_cast<const bf16*>(d.W0) + o0 * I);
+    const uint4* x = reinterpret_cast<const uint4*>(d.X);
+    const int r = (int)d.rank;
+    const bf16* U = static_cast<const bf16*>(d.U);
+    const float* Tp = T + (int64_t)p * M * g.rmax;
+    // the rank term and the row scales first: their loads overlap the sweep's
+    float y[kGroupRows][M], sv[kGroupRows];
+#pragma unroll
+    for (int k = 0; k < kGroupRows; ++k) {
+      sv[k] = k < nb ? __ldg(d.s + o0 + k) : 0.f;
+#pragma unroll
+      for (int m = 0; m < M; ++m) y[k][m] = 0.f;
+    }
+    for (int j = lane; j < r; j += 32) {
+      float t[M];
+#pragma unroll
+      for (int m = 0; m < M; ++m) t[m] = Tp[m * r + j];
+#pragma unroll
+      for (int k = 0; k < kGroupRows; ++k) {
+        if (k >= nb) break;
+        const float u = __bfloat162float(U[(o0 + k) * r + j]);
+#pragma unroll
+        for (int m = 0; m < M; ++m) y[k][m] = fmaf(u, t[m], y[k][m]);
+      }
+    }
+    uint64_t acc[kGroupRows][M];
+#pragma unroll
+    for (int k = 0; k < kGroupRows; ++k)
+#pragma unroll
+      for (int m = 0; m < M; ++m) acc[k][m] = 0;
+    for (int64_t v0 = lane; v0 < nv; v0 += 32 * kGroupUnroll) {
+      uint4 wv[kGroupUnroll][kGroupRows];
+#pragma unroll
+      for (int u = 0; u < kGroupUnroll; ++u) {
+        const int64_t v = v0 + 32 * u;
+#pragma unroll
+        for (int k = 0; k < kGroupRows; ++k)
+          wv[u][k] = (v < nv && k < nb) ? __ldcs(w + k * nv + v) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kGroupUnroll; ++u) {
+        const int64_t v = v0 + 32 * u;
+        if (v >= nv) break;
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+          uint64_t px[4];
+          bf16x8_to_f32x2(__ldg(x + m * nv + v), px);
+#pragma unroll
+          for (int k = 0; k < kGroupRows; ++k) {
+            uint64_t pw[4];
+            bf16x8_to_f32x2(wv[u][k], pw);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) fma_f32x2(acc[k][m], pw[q], px[q]);
+          }
+        }
+      }
+    }
+    // Y = s * dot + rank term, one warp reduction per row and token
+#pragma unroll
+    for (int k = 0; k < kGroupRows; ++k) {
+      if (k >= nb) break;
+#pragma unroll
+      for (int m = 0; m < M; ++m) {
+        const float yk = warp_sum(fmaf(sv[k], sum_f32x2(acc[k][m]), y[k][m]));
+        if (lane == m) static_cast<bf16*>(d.Y)[m * d.O + o0 + k] = __float2bfloat16_rn(yk);
+      }
+    }
+    row += nb;
   }
 }
 
@@ -422,7 +613,9 @@ cudaError_t launch_m(const LaunchCtx& c, GemvArgs a, const void* V) {
   // the fewest rows per warp that keep every CTA resident in one wave
   const int64_t capacity = (int64_t)c.num_sms * resident_ctas<M, FP4>(c.device, smem) * kWarps;
   a.rpw = (int)ceil_div(a.O, capacity);
-  const int64_t grid = ceil_div(a.O, (int64_t)kWarps * a.rpw);
+  // NVFP4 splits the rows evenly over one full wave; bf16 gives every warp rpw
+  const int64_t grid = FP4 ? std::min(capacity / kWarps, ceil_div(a.O, (int64_t)kWarps))
+                           : ceil_div(a.O, (int64_t)kWarps * a.rpw);
   return launch_pdl(gemv_rows_kernel<M, FP4>, dim3((unsigned)grid), dim3(kThreads), smem, c.stream, 1, a);
 }
 
@@ -432,6 +625,51 @@ int forward_gemv_max_tokens() { return kMaxTokens; }
 
 size_t forward_gemv_workspace_bytes(int64_t M, int r) {
   return (M >= 1 && M <= kMaxTokens && r > 0) ? (size_t)kXvParts * M * r * sizeof(float) : 0;
+}
+
+size_t forward_grouped_workspace_bytes(int count, int64_t M, int rmax) {
+  return rmax > 0 ? (size_t)count * M * rmax * sizeof(float) * (kGroupParts + 1) : 0;
+}
+
+bool launch_forward_grouped(const LaunchCtx& c, const theta_forward_problem* host, const theta_forward_problem* dev,
+                            int count, int64_t M, int rmax, void* ws, cudaError_t* e) {
+  *e = cudaSuccess;
+  if (M < 1 || M > kMaxTokens || count < 1 || count > kMaxGroup || rmax > kMaxRank) return false;
+  GroupArgs g = {};
+  g.P = dev;
+  g.count = count;
+  g.rmax = rmax;
+  g.prefix[0] = 0;
+  g.elems[0] = 0;
+  for (int i = 0; i < count; ++i) {
+    if (g.prefix[i] + host[i].O > INT32_MAX) return false;
+    g.prefix[i + 1] = (int32_t)(g.prefix[i] + host[i].O);
+    g.elems[i + 1] = g.elems[i] + host[i].O * host[i].I;
+  }
+  float* parts = static_cast<float*>(ws);
+  float* T = parts + (size_t)count * kGroupParts * M * rmax;
+  g.T = T;
+  if (rmax > 0) {
+    *e = M == 1 ? launch_pdl(grouped_xv_kernel<1>, dim3(kGroupParts, (unsigned)count), dim3(kThreads), 0, c.stream, 1,
+                             dev, rmax, parts)
+                : launch_pdl(grouped_xv_kernel<2>, dim3(kGroupParts, (unsigned)count), dim3(kThreads), 0, c.stream, 1,
+                             dev, rmax, parts);
+    if (*e != cudaSuccess) return true;
+    *e = M == 1 ? launch_pdl(grouped_t_kernel<1>, dim3((unsigned)count), dim3(kThreads), 0, c.stream, 1, dev, rmax,
+                             (const float*)parts, T)
+                : launch_pdl(grouped_t_kernel<2>, dim3((unsigned)count), dim3(kThreads), 0, c.stream, 1, dev, rmax,
+                             (const float*)parts, T);
+    if (*e != cudaSuccess) return true;
+  }
+  auto go = [&](auto kern) {
+    static int cached[2][64] = {};
+    int& n = cached[M - 1][c.device];
+    if (!n && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, 0) != cudaSuccess || n < 1)) n = 1;
+    const int64_t grid = std::min((int64_t)c.num_sms * n, ceil_div((int64_t)g.prefix[count], (int64_t)kWarps));
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), 0, c.stream, 1, g);
+  };
+  *e = M == 1 ? go(grouped_rows_kernel<1>) : go(grouped_rows_kernel<2>);
+  return true;
 }
 
 bool launch_forward_gemv(const LaunchCtx& c, const void* X, const void* W0, const float* s, const void* U,

@@ -67,6 +67,11 @@ bool launch_forward_gemv(const LaunchCtx& c, const void* X, const void* W0, cons
 cudaError_t launch_nvfp4_quantize(const LaunchCtx& c, const void* W, int64_t O, int64_t I, void* codes, void* scales,
                                   float* g, void* ws);
 size_t forward_nvfp4_workspace_bytes(int64_t M, int64_t I, int r);
+// Grouped few-token forward over a problem table (host copy for sizes, device
+// copy for the kernels); rmax = the largest rank. false: outside its range.
+size_t forward_grouped_workspace_bytes(int count, int64_t M, int rmax);
+bool launch_forward_grouped(const LaunchCtx& c, const theta_forward_problem* host, const theta_forward_problem* dev,
+                            int count, int64_t M, int rmax, void* ws, cudaError_t* e);
 bool launch_forward_nvfp4(const LaunchCtx& c, const void* X, const void* codes, const void* scales, const float* g,
                           const float* s, const void* U, const void* V, int64_t M, int64_t O, int64_t I, int r,
                           void* Y, void* ws, cudaError_t* e);

@@ -4,6 +4,7 @@
 // rejected call leaves device memory untouched. Kernels run on the caller's
 // stream; nothing here allocates device memory or synchronises (except
 // theta_device_status, whose job is to synchronise).
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -310,6 +311,47 @@ THETA_API int theta_linear_forward(const void* X, int64_t M, int64_t I, const vo
   return THETA_OK;
 }
 
+THETA_API int theta_linear_forward_grouped(const theta_forward_problem* problems,
+                                           const theta_forward_problem* problems_device, int count, int64_t M,
+                                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (!problems || !problems_device)
+    return fail(THETA_ERR_INVALID_ARG, "theta_linear_forward_grouped: NULL problem table");
+  if (count < 1 || count > THETA_MAX_GROUP)
+    return fail(THETA_ERR_INVALID_ARG, "theta_linear_forward_grouped: count %d outside [1, %d]", count,
+                THETA_MAX_GROUP);
+  if (M < 1) return fail(THETA_ERR_INVALID_ARG, "theta_linear_forward_grouped: M < 1");
+  if (M > 2) return fail(THETA_ERR_UNSUPPORTED, "theta_linear_forward_grouped: one or two tokens only");
+  if (reinterpret_cast<uintptr_t>(problems_device) % alignof(theta_forward_problem))
+    return fail(THETA_ERR_ALIGNMENT, "theta_linear_forward_grouped: misaligned device problem table");
+  int rmax = 0;
+  for (int i = 0; i < count; ++i) {
+    const theta_forward_problem& p = problems[i];
+    if (p.O < 1 || p.I < 1 || p.rank < 0 || p.rank > 256)
+      return fail(THETA_ERR_INVALID_ARG, "theta_linear_forward_grouped: problem %d: need O, I >= 1, 0 <= rank <= 256",
+                  i);
+    if (!p.X || !p.W0 || !p.s || !p.Y || (p.rank > 0 && (!p.U || !p.V)))
+      return fail(THETA_ERR_INVALID_ARG, "theta_linear_forward_grouped: problem %d: NULL pointer", i);
+    if (!aligned16(p.X) || !aligned16(p.W0) || !aligned16(p.s) ||
+        (p.rank > 0 && (!aligned16(p.U) || !aligned16(p.V))) || p.I % 8 || p.O % 8 || p.rank % 8)
+      return fail(THETA_ERR_ALIGNMENT,
+                  "theta_linear_forward_grouped: problem %d: 16-byte aligned pointers and I, O, rank multiples of 8",
+                  i);
+    rmax = std::max(rmax, (int)p.rank);
+  }
+  const size_t need = forward_grouped_workspace_bytes(count, M, rmax);
+  if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return fail(THETA_ERR_WORKSPACE, "theta_linear_forward_grouped: need %zu bytes of 16-byte aligned workspace",
+                need);
+  LaunchCtx c;
+  int st = make_ctx(stream, &c);
+  if (st) return st;
+  cudaError_t ce = cudaSuccess;
+  if (!launch_forward_grouped(c, problems, problems_device, count, M, rmax, workspace, &ce))
+    return fail(THETA_ERR_UNSUPPORTED, "theta_linear_forward_grouped: outside the grouped sweep");
+  if (ce != cudaSuccess) return fail_cuda(ce, "theta_linear_forward_grouped launch");
+  return THETA_OK;
+}
+
 THETA_API int theta_linear_gate_up_forward(const void* X, int64_t M, int64_t I, int64_t O, int rank,
                                            theta_dtype dt, const void* W0_gate, const float* s_gate,
                                            const void* U_gate, const void* V_gate, const void* W0_up,
@@ -432,6 +474,11 @@ THETA_API int theta_workspace_size(int op, int64_t M, int64_t O, int64_t I, int 
     case THETA_OP_LINEAR_FORWARD_NVFP4:
       if (M < 1 || rank < 0 || I < 1) return fail(THETA_ERR_INVALID_ARG, "theta_workspace_size: bad M, I or rank");
       *bytes = forward_nvfp4_workspace_bytes(M, I, rank);
+      return THETA_OK;
+    case THETA_OP_LINEAR_FORWARD_GROUPED:  // O carries the problem count, rank the largest rank
+      if (M < 1 || M > 2 || O < 1 || O > THETA_MAX_GROUP || rank < 0 || rank > 256)
+        return fail(THETA_ERR_INVALID_ARG, "theta_workspace_size: bad M, count or rank for the grouped forward");
+      *bytes = forward_grouped_workspace_bytes((int)O, M, rank);
       return THETA_OK;
     case THETA_OP_RESIDUAL_SVD:  // M carries the number of samples
       if (M < 1 || rank < 1 || M < rank || O < 1 || I < 1)

@@ -364,7 +364,7 @@ def check_nvfp4(o):
                        rtol=1e-13, atol=1e-13)
 
 
-# --------------------------------------------------------------- pipeline# --------------------------------------------------------------- pipeline# --------------------------------------------------------------- pipeline
+# --------------------------------------------------------------- pipeline
 def check_decompose(o):
     rng = _rng(9)
     L, O, I = 4, 6, 10

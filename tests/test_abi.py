@@ -110,6 +110,39 @@ def test_nvfp4_validation(lib):
     assert lib.theta_workspace_size(lib.THETA_OP_NVFP4_QUANTIZE, 1, 8, 64, 0, lib.THETA_BF16) == 16
 
 
+def test_grouped_forward_validation(lib):
+    raw = lib.lib
+    P = lib.theta_forward_problem
+    p = 4096  # a 16-byte aligned fake device address: validation fails before any launch
+
+    def table(*probs):
+        arr = (P * len(probs))(*probs)
+        return ctypes.cast(arr, ctypes.c_void_p), arr
+
+    good = P(p, p, p, p, p, p, 64, 128, 16)
+    h, keep = table(good, P(p, p, p, None, None, p, 8, 8, 0))
+    d = ctypes.c_void_p(p)
+    assert ctypes.sizeof(P) == 72
+    assert raw.theta_linear_forward_grouped(None, d, 2, 1, d, 1 << 20, None) == -1          # no host table
+    assert raw.theta_linear_forward_grouped(h, d, 0, 1, d, 1 << 20, None) == -1             # count 0
+    assert raw.theta_linear_forward_grouped(h, d, 257, 1, d, 1 << 20, None) == -1           # count > max
+    assert raw.theta_linear_forward_grouped(h, d, 2, 3, d, 1 << 20, None) == -2             # M > 2
+    assert raw.theta_linear_forward_grouped(h, ctypes.c_void_p(p + 4), 2, 1, d, 1 << 20, None) == -3
+    assert raw.theta_linear_forward_grouped(h, d, 2, 1, None, 0, None) == -6                # no workspace
+    need = lib.theta_workspace_size(lib.THETA_OP_LINEAR_FORWARD_GROUPED, 1, 2, 0, 16, lib.THETA_BF16)
+    assert need == 2 * 16 * 4 * 9
+    assert raw.theta_linear_forward_grouped(h, d, 2, 1, d, need - 1, None) == -6
+    h2, keep2 = table(good, P(p, p, p, p, p, p, 64, 128, 12))                               # rank % 8
+    assert raw.theta_linear_forward_grouped(h2, d, 2, 1, d, 1 << 20, None) == -3
+    h3, keep3 = table(good, P(p, p, p, None, p, p, 64, 128, 8))                             # rank > 0, no U
+    assert raw.theta_linear_forward_grouped(h3, d, 2, 1, d, 1 << 20, None) == -1
+    h4, keep4 = table(P(p + 2, p, p, p, p, p, 64, 128, 16))                                 # X misaligned
+    assert raw.theta_linear_forward_grouped(h4, d, 1, 1, d, 1 << 20, None) == -3
+    assert lib.theta_workspace_size(lib.THETA_OP_LINEAR_FORWARD_GROUPED, 2, 1, 0, 0, lib.THETA_BF16) == 0
+    with pytest.raises(lib.ThetaError):
+        lib.theta_workspace_size(lib.THETA_OP_LINEAR_FORWARD_GROUPED, 3, 1, 0, 0, lib.THETA_BF16)
+
+
 def test_residual_svd_validation(lib):
     raw = lib.lib
     p = ctypes.c_void_p(16)
