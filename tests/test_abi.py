@@ -143,6 +143,19 @@ def test_grouped_forward_validation(lib):
         lib.theta_workspace_size(lib.THETA_OP_LINEAR_FORWARD_GROUPED, 3, 1, 0, 0, lib.THETA_BF16)
 
 
+def test_forward_problem_layout(lib):
+    """The binding's struct matches theta_forward_problem field for field:
+    six pointers, then O, I, rank as int64, 72 bytes in the header's order."""
+    text = open(HEADER).read()
+    body = re.search(r"typedef struct theta_forward_problem \{(.*?)\} theta_forward_problem;", text, re.S).group(1)
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = re.findall(r"\b(\w+);", body)
+    P = lib.theta_forward_problem
+    assert fields == [name for name, _ in P._fields_]
+    assert [getattr(P, name).offset for name in fields] == [0, 8, 16, 24, 32, 40, 48, 56, 64]
+    assert ctypes.sizeof(P) == 72 and ctypes.alignment(P) == 8
+
+
 def test_residual_svd_validation(lib):
     raw = lib.lib
     p = ctypes.c_void_p(16)
