@@ -822,7 +822,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of replaying CUDA graphs")
-    ap.add_argument("--streams", type=int, default=16, help="streams the independent calls of a stage spread over")
+    ap.add_argument("--streams", type=int, default=32, help="streams the independent calls of a stage spread over")
     ap.add_argument("--per-call-decode", action="store_true",
                     help="one theta_linear_forward per problem for one or two tokens instead of a grouped call")
     ap.add_argument("--skip-e2e", action="store_true")

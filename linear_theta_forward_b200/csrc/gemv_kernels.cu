@@ -416,8 +416,8 @@ __global__ void __launch_bounds__(kThreads) gemv_rows_kernel(const __grid_consta
 // the row widths); a warp owns a contiguous range of those rows and takes
 // them kGroupRows at a time (dot products, rank terms, Y).
 constexpr int kGroupParts = 8;
-constexpr int kGroupRows = 4;    // rows of one problem a warp takes at a time
-constexpr int kGroupUnroll = 2;  // 16-byte loads per row in flight per lane
+constexpr int kGroupRows = 2;    // rows of one problem a warp takes at a time
+constexpr int kGroupUnroll = 4;  // 16-byte loads per row in flight per lane
 constexpr int kMaxGroup = THETA_MAX_GROUP;
 
 struct GroupArgs {
