@@ -7,7 +7,7 @@
 // W0 and each of its warps every eighth row of it, so at any moment a CTA
 // reads eight consecutive rows -- one compact window of memory that moves
 // front to back, the access pattern that sustains the most read bandwidth
-// (tile kernels instead walk 128-row column strips). A lane keeps UNR
+// (tile kernels instead walk 128-row column strips). A lane keeps kUnroll
 // 16-byte loads of its row in flight; X (a few KB, shared by every CTA)
 // comes through L1. All CTAs are resident at once and every warp has the
 // same number of rows, so they finish together.
@@ -24,9 +24,13 @@
 //
 // The same sweep also reads the shared block in NVFP4 (codes, E4M3 block
 // scales, fp32 tensor scale; the format the pages weigh in "Quality" -- what
-// NVFP4 quantization costs): 0.5625 bytes per weight instead of 2. Its rows are split evenly over one full wave of CTAs, each
-// warp taking a contiguous range; see the FP4 branch of gemv_rows_kernel.
-// The encoder (nvfp4_amax_kernel, nvfp4_quant_kernel) sits at the end.
+// NVFP4 quantization costs): 0.5625 bytes per weight instead of 2. Its rows
+// are split evenly over one full wave of CTAs, each warp taking a
+// contiguous range; see the FP4 branch of gemv_rows_kernel. The encoder
+// (nvfp4_amax_kernel, nvfp4_quant_kernel) sits at the end.
+//
+// The grouped kernels (grouped_*_kernel) run many such forwards -- every
+// family of every layer of a decode step -- as one sweep over all their rows.
 #include <cuda_fp16.h>
 
 #include <algorithm>
