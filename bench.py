@@ -453,6 +453,7 @@ def run_reference(args):
     line = result_line(value=value, unit="GB/s", n_gpus=args.gpus, steps=args.steps, warmup=args.warmup,
                        ms_per_step=per_step * 1e3, extra={
                            "impl": "reference", "dtype": "f64",
+                           "data": "synthetic (seeded; weights, factors and activations drawn on the host)",
                            "config": {"workload": WORKLOAD, "sample_rows_per_family": args.ref_rows,
                                       "l2": "n/a (CPU)"},
                            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
