@@ -328,9 +328,9 @@ int theta_linear_forward_grouped(const theta_forward_problem* problems, const th
  * group's power of two, and the row sum multiplied by g.
  *   X [M, I], U [O, rank], V [I, rank], Y [M, O] bf16; s fp32 [O]; codes,
  *   scales, g as written by theta_nvfp4_quantize. M <= 2 (else
- *   THETA_ERR_UNSUPPORTED); I a multiple of 32 and at most 49152 for one
- *   token, 24576 for two (X must fit in shared memory; else
- *   THETA_ERR_UNSUPPORTED); O, rank multiples of 8.
+ *   THETA_ERR_UNSUPPORTED); I a multiple of 32 with M * ceil(I / 1024) <= 99
+ *   (X in fp16 must fit in shared memory: I <= 101376 for one token, 50176
+ *   for two; else THETA_ERR_UNSUPPORTED); O, rank multiples of 8.
  *   workspace: theta_workspace_size(THETA_OP_LINEAR_FORWARD_NVFP4, M, O, I,
  *   rank, THETA_BF16) bytes (the partial sums of T = X.V; 0 at rank 0).
  */
