@@ -110,3 +110,12 @@ def test_gemma3_1b_layers(lib, torch, M):
         lib.theta_linear_forward(X, W0, s, U, V, Y1, fws)
         d = (Y.float() - Y1.float()).abs().max().item()
         assert d <= 2 ** -7 * Y1.float().abs().max().item(), f"problem {k}: grouped vs single {d}"
+
+
+def test_max_count_two_tokens(lib, torch):
+    """256 problems of two tokens, widths 8..40 rows, ranks 0/8/16."""
+    X = syn.host_activations(2, 64, seed=12, tag="grouped-many2", dtype="bf16")
+    hosts = [host_problem(2, 8 * (1 + k % 5), 64, 8 * (k % 3), 300 + k, X=X) for k in range(256)]
+    _, Ys = run_group(lib, torch, hosts, 2)
+    for k, ((X_, W0, s, U, V), Y) in enumerate(zip(hosts, Ys)):
+        assert_close(Y, oracle.linear_forward(*oracle_args(X_, W0, s, U, V)), "bf16", f"problem {k} of 256, M=2")

@@ -126,3 +126,40 @@ def test_forward_token_scales(lib, torch, xs):
     ref = oracle.linear_forward_nvfp4(X, host(codes), host(scales), host(g)[0], s, U, V)
     for m in range(M):  # each token against its own scale
         assert_close(host(Y)[m:m + 1].astype(np.float64), ref[m:m + 1], "bf16", f"token {m} x{xs:g}")
+
+
+@pytest.mark.parametrize("M,I", [(1, 101376), (2, 50176)])
+def test_forward_at_shared_memory_limit(lib, torch, M, I):
+    """The widest rows the sweep takes: X in fp16 for M tokens fills 200 KB
+    of shared memory (M * ceil(I / 1024) = 99 or 98 groups)."""
+    O, r = 64, 8
+    W0 = syn.host_normal((O, I), 0.02, 9, "W0wide", O, I, dtype="bf16")
+    X = syn.host_activations(M, I, seed=9, tag="nvfp4wide", dtype="bf16")
+    s = (1.0 + syn.host_normal((O,), 0.05, 9, "s", O)).astype(np.float32)
+    U = syn.host_normal((O, r), 0.01, 9, "U", O, r, dtype="bf16")
+    V = syn.host_normal((I, r), 0.01, 9, "V", I, r, dtype="bf16")
+    codes, scales, g = encode(lib, torch, dev(W0, "bf16"))
+    Y = torch.empty(M, O, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(lib.theta_workspace_size(lib.THETA_OP_LINEAR_FORWARD_NVFP4, M, O, I, r, lib.THETA_BF16),
+                     dtype=torch.uint8, device="cuda")
+    lib.theta_linear_forward_nvfp4(dev(X, "bf16"), codes, scales, g, dev(s, "f32"), dev(U, "bf16"), dev(V, "bf16"),
+                                   Y, ws)
+    lib.theta_device_status()
+    ref = oracle.linear_forward_nvfp4(X, host(codes), host(scales), host(g)[0], s, U, V)
+    assert_close(host(Y), ref, "bf16", f"Y M={M} I={I}")
+
+
+def test_forward_past_shared_memory_limit_is_refused(lib, torch):
+    """One group more than shared memory holds: THETA_ERR_UNSUPPORTED before
+    any launch, and the device stays clean."""
+    M, O, I = 1, 8, 102400
+    codes = torch.zeros(O, I // 2, dtype=torch.uint8, device="cuda")
+    scales = torch.zeros(O, I // 16, dtype=torch.uint8, device="cuda")
+    g = torch.ones(1, dtype=torch.float32, device="cuda")
+    X = torch.zeros(M, I, dtype=torch.bfloat16, device="cuda")
+    s = torch.ones(O, dtype=torch.float32, device="cuda")
+    Y = torch.empty(M, O, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(lib.ThetaError) as err:
+        lib.theta_linear_forward_nvfp4(X, codes, scales, g, s, None, None, Y, None)
+    assert err.value.status == -2
+    lib.theta_device_status()
