@@ -346,9 +346,9 @@ int theta_linear_forward_nvfp4(const void* X, int64_t M, int64_t I, const void* 
  * Same arguments, arithmetic, kernels and result as theta_linear_forward,
  * minus the workspace: its scratch (T = X.V) lives in a 4 MiB array built
  * into the library. It is meant for code that must not call cudaMalloc:
- * work recorded into a CUDA graph (allocation is not allowed during stream
- * capture), engines whose device memory is all owned by their own fixed
- * pool, and plugins that are handed only input and output buffers.
+ * serving engines whose device memory is all owned by their own fixed pool,
+ * with nothing left over for a library, and plugins that are handed only
+ * their input and output buffers.
  *
  *   - Capacity: the call needs theta_workspace_size(THETA_OP_LINEAR_FORWARD)
  *     bytes, at most 4 MiB (about M * rank <= 1,048,576). Larger requests

@@ -586,6 +586,7 @@ size_t fp4_smem_bytes(int64_t M, int64_t I) {
 // shared memory (registers, threads and shared memory decide).
 template <int M, bool FP4>
 int resident_ctas(int device, size_t smem) {
+  std::lock_guard<std::mutex> lk(setup_mutex());
   static int cached[64] = {};
   static size_t cached_smem[64] = {};
   if (!cached[device] || cached_smem[device] != smem) {
@@ -667,8 +668,15 @@ bool launch_forward_grouped(const LaunchCtx& c, const theta_forward_problem* hos
   }
   auto go = [&](auto kern) {
     static int cached[2][64] = {};
-    int& n = cached[M - 1][c.device];
-    if (!n && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, 0) != cudaSuccess || n < 1)) n = 1;
+    int n = 0;
+    {
+      std::lock_guard<std::mutex> lk(setup_mutex());
+      int& slot = cached[M - 1][c.device];
+      if (!slot && (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&slot, kern, kThreads, 0) != cudaSuccess ||
+                    slot < 1))
+        slot = 1;
+      n = slot;
+    }
     const int64_t grid = std::min((int64_t)c.num_sms * n, ceil_div((int64_t)g.prefix[count], (int64_t)kWarps));
     return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), 0, c.stream, 1, g);
   };

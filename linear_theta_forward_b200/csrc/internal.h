@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "theta.h"
 
 namespace theta {
@@ -16,6 +18,12 @@ struct LaunchCtx {
   int device;
   int policy;  // theta_policy at the time of the call
 };
+
+// Held while a kernel's one-time, per-device set-up (attributes, occupancy
+// and cluster queries, the caches that remember them) runs, so that threads
+// making their first calls at once neither race on a cache nor read one that
+// is half written.
+std::mutex& setup_mutex();
 
 // ---- streaming kernels (stream_kernels.cu)
 cudaError_t launch_band_mean(const LaunchCtx& c, theta_dtype dt, const void* const* w, int n,
@@ -40,7 +48,10 @@ size_t frob_workspace_bytes();
 cudaError_t launch_frob(const LaunchCtx& c, theta_dtype dt, const void* a, const void* b,
                         int64_t n, double* out, void* ws);
 
-// ---- CUDA-core GEMM paths (simt_kernels.cu): fp32 forward / reconstruct
+// ---- CUDA-core GEMM paths (simt_kernels.cu): fp32 forward / reconstruct.
+// Output tiles are 64 x 64; the grid's y extent (tiles of M for the forward,
+// of O for reconstruct) is limited to 65535, so callers refuse larger sizes.
+constexpr int64_t kSimtMaxRows = (int64_t)65535 * 64;
 cudaError_t launch_xv_simt(const LaunchCtx& c, theta_dtype dt, const void* X, const void* V,
                            int64_t M, int64_t I, int r, float* T);
 cudaError_t launch_forward_simt(const LaunchCtx& c, theta_dtype dt, const void* X,

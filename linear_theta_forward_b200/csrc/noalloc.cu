@@ -5,11 +5,10 @@
 // (the one- and two-token path keeps 16 fp32 partial sums of T instead,
 // 64 * M * rank bytes, at most 32 KB).
 // Most callers pass a buffer they allocated once. Some cannot allocate at
-// all: code that records a CUDA graph (cudaMalloc is not allowed while a
-// stream is being captured), engines whose device memory is handed out by
-// their own fixed pool with nothing left for a library, and plugins that are
-// given only input and output pointers. This entry point serves them from a
-// fixed array compiled into the library.
+// all: engines whose device memory is handed out by their own fixed pool
+// with nothing left for a library, and plugins that are given only input and
+// output pointers. This entry point serves them from a fixed array compiled
+// into the library.
 //
 // The array below is ordinary device memory of the module: every GPU that
 // loads the library holds it, kScratchBytes of it, until the process exits.

@@ -518,12 +518,14 @@ template <typename T, bool BAND, int TPR, int VPT>
 cudaError_t launch_one(const LaunchCtx& c, const PreludeArgs& a, int grid, size_t smem) {
   auto kern = prelude_pipe_kernel<T, BAND, TPR, VPT>;
   static bool opted[64] = {};
+  std::unique_lock<std::mutex> lk(setup_mutex());
   if (!opted[c.device]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemBudget + 128 + 2 * kMaxSlots * 8);
     if (e != cudaSuccess) return e;
     opted[c.device] = true;
   }
+  lk.unlock();
   return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), smem, c.stream, 1, a);
 }
 
@@ -636,6 +638,7 @@ template <typename T, int TPR, int VPT, int LPI>
 cudaError_t launch_two(const LaunchCtx& c, const PreludeArgs& a, int grid, size_t smem) {
   auto kern = prelude_band2_kernel<T, TPR, VPT, LPI>;
   static int resident[64] = {};  // CTAs per SM (registers and shared memory decide)
+  std::unique_lock<std::mutex> lk(setup_mutex());
   if (!resident[c.device]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemBudget + 128 + 2 * kMaxSlots * 8);
@@ -645,8 +648,10 @@ cudaError_t launch_two(const LaunchCtx& c, const PreludeArgs& a, int grid, size_
     if (e != cudaSuccess) return e;
     resident[c.device] = n < 1 ? 1 : n;
   }
+  const int per_sm = resident[c.device];
+  lk.unlock();
   // one wave: a CTA that waited for a slot of the SM would start its units late
-  if (grid > c.num_sms * resident[c.device]) grid = c.num_sms * resident[c.device];
+  if (grid > c.num_sms * per_sm) grid = c.num_sms * per_sm;
   return launch_pdl(kern, dim3((unsigned)grid), dim3(kThreads), smem, c.stream, 1, a);
 }
 

@@ -416,6 +416,7 @@ cudaError_t gemm(const LaunchCtx& c, const TA* A, const TB* B, int64_t M, int64_
 }
 
 cudaError_t small_kernels_ready(int device) {
+  std::lock_guard<std::mutex> lk(setup_mutex());
   static bool done[64] = {};
   if (done[device]) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(chol_inv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

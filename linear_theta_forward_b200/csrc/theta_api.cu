@@ -93,6 +93,11 @@ size_t forward_ws_bytes(int64_t M, int r, theta_dtype dt) {
 
 }  // namespace
 
+std::mutex& setup_mutex() {
+  static std::mutex mu;
+  return mu;
+}
+
 // Lets other translation units report through theta_last_error().
 int report_error(int status, const char* message) {
   t_last_error = message;
@@ -246,13 +251,18 @@ THETA_API int theta_reconstruct(const float* s, const void* W0, const void* U, c
     return fail(THETA_ERR_INVALID_ARG, "theta_reconstruct: need O, I >= 1 and rank >= 0");
   if (!s || !W0 || !W_out || (rank > 0 && (!U || !V)))
     return fail(THETA_ERR_INVALID_ARG, "theta_reconstruct: NULL pointer");
-  LaunchCtx c;
-  int st = make_ctx(stream, &c);
-  if (st) return st;
   if (dt == THETA_BF16) {
     if (!aligned16(s) || !aligned16(W0) || !aligned16(W_out) || (rank > 0 && (!aligned16(U) || !aligned16(V))) ||
         I % 8 || rank % 8)
       return fail(THETA_ERR_ALIGNMENT, "theta_reconstruct: bf16 needs 16-byte aligned pointers and I, rank multiples of 8");
+  } else if (O > kSimtMaxRows) {
+    return fail(THETA_ERR_UNSUPPORTED, "theta_reconstruct: fp32 path takes at most %lld rows",
+                (long long)kSimtMaxRows);
+  }
+  LaunchCtx c;
+  int st = make_ctx(stream, &c);
+  if (st) return st;
+  if (dt == THETA_BF16) {
     cudaError_t ce = cudaSuccess;
     st = launch_reconstruct_umma(c, s, W0, U, V, O, I, rank, W_out, &ce);
     if (st == THETA_ERR_CUDA) return fail_cuda(ce, "theta_reconstruct (tensor-core path)");
@@ -292,14 +302,22 @@ THETA_API int theta_linear_forward(const void* X, int64_t M, int64_t I, const vo
   const size_t need = forward_ws_bytes(M, rank, dt);
   if (need && (!workspace || workspace_bytes < need || !aligned16(workspace)))
     return fail(THETA_ERR_WORKSPACE, "theta_linear_forward: need %zu bytes of 16-byte aligned workspace", need);
-  LaunchCtx c;
-  int st = make_ctx(stream, &c);
-  if (st) return st;
   if (dt == THETA_BF16) {
     if (!aligned16(X) || !aligned16(W0) || !aligned16(Y) || !aligned16(s) ||
         (rank > 0 && (!aligned16(U) || !aligned16(V))) || I % 8 || O % 8 || rank % 8)
       return fail(THETA_ERR_ALIGNMENT,
                   "theta_linear_forward: bf16 needs 16-byte aligned pointers and I, O, rank multiples of 8");
+    if (rank > 0 && (M + 127) / 128 > 65535)
+      return fail(THETA_ERR_UNSUPPORTED, "theta_linear_forward: bf16 with rank > 0 takes at most %lld tokens",
+                  (long long)65535 * 128);
+  } else if (M > kSimtMaxRows) {
+    return fail(THETA_ERR_UNSUPPORTED, "theta_linear_forward: fp32 path takes at most %lld tokens",
+                (long long)kSimtMaxRows);
+  }
+  LaunchCtx c;
+  int st = make_ctx(stream, &c);
+  if (st) return st;
+  if (dt == THETA_BF16) {
     cudaError_t ce = cudaSuccess;
     st = launch_forward_umma(c, X, W0, s, U, V, M, O, I, rank, Y, workspace, &ce);
     if (st == THETA_ERR_CUDA) return fail_cuda(ce, "theta_linear_forward (tensor-core path)");
@@ -377,6 +395,9 @@ THETA_API int theta_linear_gate_up_forward(const void* X, int64_t M, int64_t I, 
       O % 8 || rank % 8)
     return fail(THETA_ERR_ALIGNMENT,
                 "theta_linear_gate_up_forward: bf16 needs 16-byte aligned pointers and I, O, rank multiples of 8");
+  if (rank > 0 && (M + 127) / 128 > 65535)
+    return fail(THETA_ERR_UNSUPPORTED, "theta_linear_gate_up_forward: rank > 0 takes at most %lld tokens",
+                (long long)65535 * 128);
   LaunchCtx c;
   int st = make_ctx(stream, &c);
   if (st) return st;

@@ -586,7 +586,9 @@ struct KernelInfo {
 };
 
 template <typename Kern>
-cudaError_t prepare_kernel(KernelInfo* info, Kern kern, int threads, int smem, int tmem_cols, bool clusters) {
+cudaError_t prepare_kernel(KernelInfo* info, int device, Kern kern, int threads, int smem, int tmem_cols,
+                           bool clusters) {
+  std::lock_guard<std::mutex> lk(setup_mutex());
   if (info->ready) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -603,9 +605,9 @@ cudaError_t prepare_kernel(KernelInfo* info, Kern kern, int threads, int smem, i
   // instructions). Tensor memory must cover all of them, or allocation
   // would stall.
   int dev_smem = 0, reserved = 0;
-  e = cudaDeviceGetAttribute(&dev_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, 0);
+  e = cudaDeviceGetAttribute(&dev_smem, cudaDevAttrMaxSharedMemoryPerMultiprocessor, device);
   if (e != cudaSuccess) return e;
-  e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, 0);
+  e = cudaDeviceGetAttribute(&reserved, cudaDevAttrReservedSharedMemoryPerBlock, device);
   if (e != cudaSuccess) return e;
   int blocks = dev_smem / (smem + reserved);
   const int by_threads = 2048 / threads;
@@ -619,7 +621,11 @@ cudaError_t prepare_kernel(KernelInfo* info, Kern kern, int threads, int smem, i
   info->blocks_per_sm = blocks;
   info->max_cluster = 1;
   if (clusters) {
-    // the largest cluster (16, else 8) that the GPU can place at all
+    // the largest cluster (16, else 8) that the GPU can place at all; a
+    // refused query sets the thread's last error, which is cleared below only
+    // when no earlier error was pending (the caller's must not be lost)
+    const bool pending = cudaPeekAtLastError() != cudaSuccess;
+    bool refused = false;
     for (int cs = 16; cs >= 8 && info->max_cluster == 1; cs /= 2) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(cs, 1, 1);
@@ -633,9 +639,11 @@ cudaError_t prepare_kernel(KernelInfo* info, Kern kern, int threads, int smem, i
       cfg.attrs = &attr;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) == cudaSuccess && n > 0) info->max_cluster = cs;
+      const cudaError_t q = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+      if (q == cudaSuccess && n > 0) info->max_cluster = cs;
+      if (q != cudaSuccess) refused = true;
     }
-    cudaGetLastError();  // a refused query above is not an error of this call
+    if (refused && !pending) cudaGetLastError();  // a refused query is not an error of this call
     if (info->max_cluster == 1) return cudaErrorInvalidConfiguration;
   }
   info->ready = true;
@@ -661,7 +669,7 @@ cudaError_t launch_tile_kernel(const LaunchCtx& c, const Maps& mp, Args args, in
   using C = Cfg<BN, MODE>;
   auto kern = umma_kernel<BN, MODE>;
   static KernelInfo info[64];
-  cudaError_t e = prepare_kernel(&info[c.device], kern, kThreads, C::kSmemBytes, C::kTmemCols, true);
+  cudaError_t e = prepare_kernel(&info[c.device], c.device, kern, kThreads, C::kSmemBytes, C::kTmemCols, true);
   if (e != cudaSuccess) return e;
   const int64_t tiles = (int64_t)m_tiles * n_tiles;
   // Tiles of 64 or more columns keep the tensor pipe busy: a second CTA on
@@ -682,7 +690,7 @@ cudaError_t launch_recon(const LaunchCtx& c, const CUtensorMap& mU, const CUtens
   using C = RecCfg<KB>;
   auto kern = recon_kernel<KB>;
   static KernelInfo info[64];
-  cudaError_t e = prepare_kernel(&info[c.device], kern, kRecThreads, C::kSmemBytes, kRecN, false);
+  cudaError_t e = prepare_kernel(&info[c.device], c.device, kern, kRecThreads, C::kSmemBytes, kRecN, false);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3((unsigned)ceil_div(I, kRecN), (unsigned)ceil_div(O, kBM), 1), dim3(kRecThreads),
                     C::kSmemBytes, c.stream, 1, mU, mV, mW0, mOut, s, O, I, c.err);
@@ -757,6 +765,8 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
   *ce = cudaSuccess;
   if (O > (int64_t)65535 * kBM || M > ((int64_t)1 << 30) || I > ((int64_t)1 << 31) - 64 || r > 256)
     return THETA_ERR_UNSUPPORTED;
+  // the T = X.V grid is one CTA row per 128 tokens (grid y <= 65535)
+  if (r > 0 && ceil_div(M, kBM) > 65535) return THETA_ERR_UNSUPPORTED;
   cudaError_t e = cudaSuccess;
   // ---- a handful of tokens: a sequential sweep over W0 on CUDA cores
   if (M <= forward_gemv_max_tokens() && launch_forward_gemv(c, X, W0, s, U, V, M, O, I, r, Y, ws, &e)) {
@@ -827,6 +837,7 @@ int launch_gate_up_umma(const LaunchCtx& c, const void* X, const void* W0g, cons
   *ce = cudaSuccess;
   if (O > (int64_t)65535 * kBM || M > ((int64_t)1 << 30) || I > ((int64_t)1 << 31) - 64 || r > 256)
     return THETA_ERR_UNSUPPORTED;
+  if (r > 0 && ceil_div(M, kBM) > 65535) return THETA_ERR_UNSUPPORTED;  // T = X.V grid height
   const size_t half = ((size_t)M * r * 2 + 255) / 256 * 256;
   bf16* t[4] = {};
   int st;

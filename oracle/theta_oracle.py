@@ -22,7 +22,7 @@ Sources (page title -- section):
   * "Quality" -- Native-equivalent at passthrough (G = num_layers rebuilds the
     weight exactly); Reconstruction error (relative Frobenius error).
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings where the pages are silent:
   * G outside [1, num_layers] is rejected.
   * W0 is the fp64 mean, rounded once to the storage dtype.
   * s is fitted against the *stored* (rounded) W0, the block the forward uses.

@@ -98,6 +98,21 @@ def test_validation_happens_before_any_cuda_call(lib):
                                             None) == -3                                          # I % 8 != 0
 
 
+def test_sizes_beyond_the_grid_limits_are_refused_on_the_host(lib):
+    """Token counts whose grids would exceed the 65535-block y extent come back
+    as THETA_ERR_UNSUPPORTED before any CUDA call (no launch error later)."""
+    raw = lib.lib
+    p = ctypes.c_void_p(256)
+    M = 65535 * 128 + 1  # one token past the T = X.V grid of the tensor-core path
+    assert raw.theta_linear_forward(p, M, 64, p, 64, p, p, p, 8, 1, p, p, 1 << 40, None) == -2
+    assert "tokens" in lib.theta_last_error()
+    assert raw.theta_linear_gate_up_forward(p, M, 64, 64, 8, 1, p, p, p, p, p, p, p, p, p, p, 1 << 40,
+                                            None) == -2
+    M32 = 65535 * 64 + 1  # past the fp32 tile grid
+    assert raw.theta_linear_forward(p, M32, 64, p, 64, p, None, None, 0, 0, p, None, 0, None) == -2
+    assert raw.theta_reconstruct(p, p, None, None, M32, 64, 0, 0, p, None) == -2
+
+
 def test_nvfp4_validation(lib):
     raw = lib.lib
     p = ctypes.c_void_p(16)
