@@ -385,10 +385,11 @@ int theta_workspace_size(int op, int64_t M, int64_t O, int64_t I, int rank, thet
  *   THETA_POLICY_LATENCY (default): when the output tiles of one call leave
  *     SMs idle, K is split over a thread-block cluster and the partial tiles
  *     are summed through distributed shared memory -- the fastest single call.
- *   THETA_POLICY_THROUGHPUT: no split; every CTA owns a whole output tile.
- *     For callers that keep the GPU busy with many independent calls on
- *     several streams, where split-K's extra CTAs, cluster scheduling and
- *     reductions cost more than they gain.
+ *   THETA_POLICY_THROUGHPUT: no split of the main projection; every CTA
+ *     owns a whole output tile. For callers that keep the GPU busy with many
+ *     independent calls on several streams, where split-K's extra CTAs,
+ *     cluster scheduling and reductions cost more than they gain. (The small
+ *     T = X.V kernel in front of it splits K under both policies.)
  * Returns THETA_ERR_INVALID_ARG for any other value. Safe to call from any
  * thread; calls already enqueued keep the policy they were launched with.
  * theta_get_policy returns the current policy.

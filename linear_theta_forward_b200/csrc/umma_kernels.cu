@@ -677,7 +677,11 @@ cudaError_t launch_tile_kernel(const LaunchCtx& c, const Maps& mp, Args args, in
   // count one CTA per SM. Narrow (decode) tiles are bound by memory latency
   // and count every co-resident CTA.
   const int capacity = c.num_sms * (BN >= 64 ? 1 : info[c.device].blocks_per_sm);
-  args.splits = c.policy == THETA_POLICY_THROUGHPUT
+  // The throughput policy gives every CTA of the main projection a whole
+  // tile. T = X.V keeps its split under both policies: it has one tile per
+  // 128 tokens, so unsplit it is a single CTA walking all of K, a serial
+  // latency chain that the forward behind it waits for.
+  args.splits = (c.policy == THETA_POLICY_THROUGHPUT && MODE != MODE_XV)
                     ? 1
                     : pick_splits(tiles, args.kb1, capacity, info[c.device].max_cluster);
   return launch_pdl(kern, dim3((unsigned)(n_tiles * args.splits), (unsigned)m_tiles, 1), dim3(kThreads), C::kSmemBytes,
