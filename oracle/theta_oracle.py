@@ -269,6 +269,26 @@ def frob_error(original, reconstructed) -> float:
     return float(num / den)
 
 
+def frob_partials(original, reconstructed):
+    """The two sums behind relative_frobenius_error ("Quality" --
+    Reconstruction error): (sum of (A - B)^2, sum of A^2) in fp64. Both are
+    plain sums over the elements, so a split of the rows into blocks gives
+    per-block sums that add up to these; the ratio of their square roots is
+    frob_error."""
+    A = np.asarray(original, dtype=F64)
+    B = np.asarray(reconstructed, dtype=F64)
+    return float(np.sum((A - B) ** 2)), float(np.sum(A ** 2))
+
+
+def frob_from_partials(num, den) -> float:
+    """sqrt(num) / sqrt(den), with the same 0/0 -> 0 and x/0 -> +inf cases as
+    frob_error."""
+    n, d = np.sqrt(F64(num)), np.sqrt(F64(den))
+    if d == 0.0:
+        return 0.0 if n == 0.0 else float("inf")
+    return float(n / d)
+
+
 # ----------------------------------------------------------------- forward
 def linear_forward(X, W0, s, U, V, out_dtype: str = "f64") -> np.ndarray:
     """Y = X·(diag(s)·W0 + U·Vᵀ)ᵀ = s ⊙ (X·W0ᵀ) + (X·V)·Uᵀ.

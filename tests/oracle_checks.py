@@ -227,6 +227,33 @@ def check_frob(o):
     assert o.frob_error(Z, np.ones((2, 2))) == float("inf")
 
 
+def check_frob_partials(o):
+    """The two sums a row-sharded error combines: hand values, the ratio they
+    give is frob_error's, and row blocks add up exactly on integer data."""
+    assert o.frob_partials(np.array([[3.0, 4.0]]), np.array([[0.0, 0.0]])) == (25.0, 25.0)
+    assert o.frob_partials(np.array([[1.0, 2.0], [2.0, 1.0]]), np.array([[1.0, 2.0], [2.0, 2.0]])) == (1.0, 10.0)
+    assert o.frob_partials(np.array([[6.0, 8.0]]), np.array([[3.0, 4.0]])) == (25.0, 100.0)
+    rng = _rng(16)
+    A = rng.standard_normal((9, 6))
+    B = A + 0.1 * rng.standard_normal((9, 6))
+    assert o.frob_from_partials(*o.frob_partials(A, B)) == o.frob_error(A, B)
+    assert o.frob_from_partials(0.0, 0.0) == 0.0 and o.frob_from_partials(2.0, 0.0) == float("inf")
+    # brute-force sums of squares by loops
+    num = sum((A[i, j] - B[i, j]) ** 2 for i in range(9) for j in range(6))
+    den = sum(A[i, j] ** 2 for i in range(9) for j in range(6))
+    n2, d2 = o.frob_partials(A, B)
+    assert math.isclose(n2, num, rel_tol=1e-14) and math.isclose(d2, den, rel_tol=1e-14)
+    # small integers: every partial sum is exact, so any split of the rows
+    # into blocks adds up to the whole bit for bit
+    Ai = rng.integers(-50, 50, size=(11, 7)).astype(np.float64)
+    Bi = rng.integers(-50, 50, size=(11, 7)).astype(np.float64)
+    whole = o.frob_partials(Ai, Bi)
+    for cuts in ([5], [1, 8], [3, 4, 9]):
+        blocks = np.split(np.arange(11), cuts)
+        parts = [o.frob_partials(Ai[b], Bi[b]) for b in blocks]
+        assert (sum(p[0] for p in parts), sum(p[1] for p in parts)) == whole
+
+
 # --------------------------------------------------------------- forward
 def check_forward(o):
     import torch
@@ -444,5 +471,5 @@ def check_gate_up(o):
 
 
 ALL_CHECKS = [check_gelu, check_gate_up, check_randomized_svd, check_nvfp4, check_round, check_bands, check_band_mean, check_row_scale, check_residual,
-              check_reconstruct, check_frob, check_forward, check_svd, check_decompose,
+              check_reconstruct, check_frob, check_frob_partials, check_forward, check_svd, check_decompose,
               check_frob_statistics]

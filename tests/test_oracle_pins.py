@@ -99,6 +99,16 @@ def _m_frob_squared(A, B):
     return e * e
 
 
+def _m_frob_partials_den_from_recon(A, B):
+    A, B = np.asarray(A, np.float64), np.asarray(B, np.float64)
+    return float(np.sum((A - B) ** 2)), float(np.sum(B ** 2))
+
+
+def _m_frob_partials_norms(A, B):
+    A, B = np.asarray(A, np.float64), np.asarray(B, np.float64)
+    return float(np.sqrt(np.sum((A - B) ** 2))), float(np.sqrt(np.sum(A ** 2)))
+
+
 def _m_forward_no_rank(X, W0, s, U, V, out_dtype="f64"):
     return oracle.linear_forward(X, W0, s, np.zeros_like(np.asarray(U, np.float64)),
                                  np.zeros_like(np.asarray(V, np.float64)), out_dtype)
@@ -194,6 +204,8 @@ MUTANTS = {
     "reconstruct_drops_scale": dict(reconstruct=_m_reconstruct_unscaled),
     "frob_normalised_by_reconstruction": dict(frob_error=_m_frob_by_recon),
     "frob_squared": dict(frob_error=_m_frob_squared),
+    "frob_partials_normalised_by_reconstruction": dict(frob_partials=_m_frob_partials_den_from_recon),
+    "frob_partials_as_norms": dict(frob_partials=_m_frob_partials_norms),
     "forward_drops_rank_term": dict(linear_forward=_m_forward_no_rank),
     "forward_scales_rank_term": dict(linear_forward=_m_forward_scale_all),
     "forward_scale_on_wrong_axis": dict(linear_forward=_m_forward_scale_rows),
