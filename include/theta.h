@@ -208,6 +208,22 @@ int theta_frob_error(const void* original, const void* reconstructed, int64_t n,
                      double* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * theta_frob_partials -- the two sums behind relative_frobenius_error
+ * ("Quality" -- Reconstruction error): out[0] = sum (A - B)^2 and
+ * out[1] = sum A^2, with the same kernels, order and precision as
+ * theta_frob_error. Both are plain sums, so when the rows of a matrix are
+ * split across GPUs (every quantity of "The theta bundle" component table is
+ * per output row) each GPU takes the sums of its rows, one all-reduce adds
+ * them, and sqrt(out[0]) / sqrt(out[1]) is the error of the whole matrix.
+ *
+ *   original, reconstructed  device [n] of dt (any shape, flattened).
+ *   out        device double[2], 8-byte aligned, written.
+ *   workspace  as for theta_frob_error (THETA_OP_FROB_ERROR).
+ */
+int theta_frob_partials(const void* original, const void* reconstructed, int64_t n, theta_dtype dt,
+                        double* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * theta_linear_forward -- the projection by the rebuilt weight without
  * forming it:  Y = X . (diag(s) . W0 + U . V^T)^T = s (.) (X . W0^T) + (X . V) . U^T
  * (identity from "The theta bundle" approximation formula).

@@ -21,7 +21,7 @@ __all__ = [
     "theta_forward_problem", "ForwardGroup", "theta_linear_forward_grouped",
     "theta_version", "theta_status_string", "theta_last_error", "theta_band_index",
     "theta_band_mean", "theta_row_scale", "theta_residual", "theta_decompose_prelude",
-    "theta_reconstruct", "theta_frob_error", "theta_linear_forward", "theta_workspace_size",
+    "theta_reconstruct", "theta_frob_error", "theta_frob_partials", "theta_linear_forward", "theta_workspace_size",
     "theta_device_status", "theta_linear_forward_noalloc", "theta_set_policy", "theta_get_policy",
     "theta_selftest_wait_timeout", "THETA_POLICY_LATENCY", "THETA_POLICY_THROUGHPUT",
 ]
@@ -55,6 +55,7 @@ _SIGNATURES = {
     "theta_decompose_prelude": (_int, _vp, _int, _int, _i64, _i64, _int, _vp, _vp, _vp, _vp),
     "theta_reconstruct": (_int, _vp, _vp, _vp, _vp, _i64, _i64, _int, _int, _vp, _vp),
     "theta_frob_error": (_int, _vp, _vp, _i64, _int, _vp, _vp, _sz, _vp),
+    "theta_frob_partials": (_int, _vp, _vp, _i64, _int, _vp, _vp, _sz, _vp),
     "theta_linear_forward": (_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp, _sz, _vp),
     "theta_linear_forward_noalloc": (_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp),
     "theta_nvfp4_quantize": (_int, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _sz, _vp),
@@ -230,6 +231,16 @@ def theta_frob_error(original, reconstructed, out, workspace, stream=None) -> No
                                 _ptr(workspace, "workspace"),
                                 workspace.numel() * workspace.element_size(), _stream(stream)),
            "theta_frob_error")
+
+
+def theta_frob_partials(original, reconstructed, out, workspace, stream=None) -> None:
+    """out: float64 CUDA tensor of two elements, receives (sum (A-B)^2,
+    sum A^2); workspace as for theta_frob_error."""
+    _check(_load().theta_frob_partials(_ptr(original, "original"), _ptr(reconstructed, "reconstructed"),
+                                   original.numel(), _dtype_code(original), _ptr(out, "out"),
+                                   _ptr(workspace, "workspace"),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)),
+           "theta_frob_partials")
 
 
 def theta_linear_forward(X, W0, s, U, V, Y, workspace=None, stream=None) -> None:

@@ -45,8 +45,9 @@ bool launch_prelude_pipe(const LaunchCtx& c, theta_dtype dt, int mode, const voi
                          const int32_t* band_start, const int32_t* band_of_layer, void* const* W0,
                          float* const* s, void* const* R, int64_t O, int64_t I, cudaError_t* e);
 size_t frob_workspace_bytes();
+// partials: out[0], out[1] receive the two sums instead of their ratio.
 cudaError_t launch_frob(const LaunchCtx& c, theta_dtype dt, const void* a, const void* b,
-                        int64_t n, double* out, void* ws);
+                        int64_t n, double* out, void* ws, bool partials = false);
 
 // ---- CUDA-core GEMM paths (simt_kernels.cu): fp32 forward / reconstruct.
 // Output tiles are 64 x 64; the grid's y extent (tiles of M for the forward,

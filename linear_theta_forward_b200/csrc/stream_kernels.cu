@@ -277,8 +277,10 @@ frob_partial_kernel(const T* __restrict__ A, const T* __restrict__ B, int64_t nv
   }
 }
 
+// Combines the block partials in a fixed order into the ratio, or (partials)
+// into the two sums themselves: out[0] = sum (A-B)^2, out[1] = sum A^2.
 __global__ void __launch_bounds__(kThreads) frob_final_kernel(const double* __restrict__ ws, int nb,
-                                                              double* __restrict__ out) {
+                                                              double* __restrict__ out, int partials) {
   pdl_enter(ws);
   double num = 0.0, den = 0.0;
   for (int k = threadIdx.x; k < nb; k += blockDim.x) {
@@ -298,6 +300,11 @@ __global__ void __launch_bounds__(kThreads) frob_final_kernel(const double* __re
     for (int k = 0; k < kThreads / 32; ++k) {
       n2 += red[k][0];
       d2 += red[k][1];
+    }
+    if (partials) {
+      out[0] = n2;
+      out[1] = d2;
+      return;
     }
     double e;
     if (d2 == 0.0)
@@ -424,7 +431,7 @@ cudaError_t residual_t(const LaunchCtx& c, const void* w, const void* W0, const 
 
 template <typename T>
 cudaError_t frob_t(const LaunchCtx& c, const void* a, const void* b, int64_t n, double* out,
-                   void* ws) {
+                   void* ws, bool partials) {
   const bool vec = aligned16(a) && aligned16(b);
   const int64_t nvec = vec ? n / Vec<T>::N : 0;
   int grid = grid_for(c, vec ? nvec : n, kThreads, 4);
@@ -433,7 +440,8 @@ cudaError_t frob_t(const LaunchCtx& c, const void* a, const void* b, int64_t n, 
   cudaError_t e = launch_pdl(frob_partial_kernel<T>, grid, kThreads, 0, c.stream, 1, static_cast<const T*>(a),
                              static_cast<const T*>(b), nvec, n, part);
   if (e != cudaSuccess) return e;
-  return launch_pdl(frob_final_kernel, 1, kThreads, 0, c.stream, 1, static_cast<const double*>(part), grid, out);
+  return launch_pdl(frob_final_kernel, 1, kThreads, 0, c.stream, 1, static_cast<const double*>(part), grid, out,
+                    partials ? 1 : 0);
 }
 
 }  // namespace
@@ -459,8 +467,9 @@ cudaError_t launch_residual(const LaunchCtx& c, theta_dtype dt, const void* w, c
 size_t frob_workspace_bytes() { return (size_t)kFrobMaxBlocks * 2 * sizeof(double); }
 
 cudaError_t launch_frob(const LaunchCtx& c, theta_dtype dt, const void* a, const void* b,
-                        int64_t n, double* out, void* ws) {
-  return dt == THETA_BF16 ? frob_t<bf16>(c, a, b, n, out, ws) : frob_t<float>(c, a, b, n, out, ws);
+                        int64_t n, double* out, void* ws, bool partials) {
+  return dt == THETA_BF16 ? frob_t<bf16>(c, a, b, n, out, ws, partials)
+                          : frob_t<float>(c, a, b, n, out, ws, partials);
 }
 
 }  // namespace theta

@@ -290,6 +290,24 @@ THETA_API int theta_frob_error(const void* original, const void* reconstructed, 
   return THETA_OK;
 }
 
+THETA_API int theta_frob_partials(const void* original, const void* reconstructed, int64_t n, theta_dtype dt,
+                                  double* out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!valid_dt(dt)) return fail(THETA_ERR_INVALID_ARG, "theta_frob_partials: bad dtype %d", (int)dt);
+  if (n < 0) return fail(THETA_ERR_INVALID_ARG, "theta_frob_partials: n < 0");
+  if ((n > 0 && (!original || !reconstructed)) || !out)
+    return fail(THETA_ERR_INVALID_ARG, "theta_frob_partials: NULL pointer");
+  if (reinterpret_cast<uintptr_t>(out) & 7u)
+    return fail(THETA_ERR_ALIGNMENT, "theta_frob_partials: out must be 8-byte aligned");
+  if (!workspace || workspace_bytes < frob_workspace_bytes() || !aligned16(workspace))
+    return fail(THETA_ERR_WORKSPACE, "theta_frob_partials: need %zu bytes of 16-byte aligned workspace",
+                frob_workspace_bytes());
+  LaunchCtx c;
+  int st = make_ctx(stream, &c);
+  if (st) return st;
+  CHECK_LAUNCH(launch_frob(c, dt, original, reconstructed, n, out, workspace, true), "theta_frob_partials launch");
+  return THETA_OK;
+}
+
 THETA_API int theta_linear_forward(const void* X, int64_t M, int64_t I, const void* W0, int64_t O,
                                    const float* s, const void* U, const void* V, int rank,
                                    theta_dtype dt, void* Y, void* workspace, size_t workspace_bytes,

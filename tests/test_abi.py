@@ -81,6 +81,9 @@ def test_validation_happens_before_any_cuda_call(lib):
     assert raw.theta_reconstruct(None, None, None, None, 8, 8, -1, 0, None, None) == -1
     assert raw.theta_frob_error(None, None, -1, 0, None, None, 0, None) == -1
     assert raw.theta_frob_error(None, None, 0, 0, ctypes.c_void_p(16), None, 0, None) == -6
+    assert raw.theta_frob_partials(None, None, -1, 0, None, None, 0, None) == -1
+    assert raw.theta_frob_partials(None, None, 0, 0, ctypes.c_void_p(12), None, 0, None) == -3   # out misaligned
+    assert raw.theta_frob_partials(None, None, 0, 0, ctypes.c_void_p(16), None, 0, None) == -6
     assert raw.theta_linear_forward(None, 0, 8, None, 8, None, None, None, 0, 0, None, None, 0, None) == -1
     assert raw.theta_linear_forward(ctypes.c_void_p(16), 4, 8, ctypes.c_void_p(16), 8, ctypes.c_void_p(16),
                                     None, None, 8, 0, ctypes.c_void_p(16), None, 0, None) == -1  # rank>0, U NULL

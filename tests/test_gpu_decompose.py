@@ -204,3 +204,47 @@ def test_frob_error_degenerate_and_closed_forms(lib, torch):
     first = out.item()
     lib.theta_frob_error(a, b, out, ws)
     assert out.item() == first
+
+
+@pytest.mark.parametrize("dt", DTYPES)
+@pytest.mark.parametrize("n", [1, 7, 1000003, 6912 * 1152])
+def test_frob_partials(lib, torch, dt, n):
+    """The two sums against the oracle's; their ratio is theta_frob_error's
+    result bit for bit (same kernels, one IEEE sqrt and division each)."""
+    import math
+    a = syn.host_normal((n,), 0.02, 2, "A", n, dtype=dt)
+    b = syn.as_dtype_values(a + syn.host_normal((n,), 0.005, 2, "B", n), dt)
+    ws = torch.empty(lib.theta_workspace_size(lib.THETA_OP_FROB_ERROR, 1, 1, 1, 0, 0), dtype=torch.uint8,
+                     device="cuda")
+    p = torch.full((2,), float("nan"), dtype=torch.float64, device="cuda")
+    out = torch.empty(1, dtype=torch.float64, device="cuda")
+    A, B = dev(a, dt), dev(b, dt)
+    lib.theta_frob_partials(A, B, p, ws)
+    lib.theta_frob_error(A, B, out, ws)
+    num, den = oracle.frob_partials(a, b)
+    g = p.cpu().tolist()
+    assert_scalar_close(g[0], num, 1e-5, "sum (A-B)^2")
+    assert_scalar_close(g[1], den, 1e-5, "sum A^2")
+    assert math.sqrt(g[0]) / math.sqrt(g[1]) == out.item()
+
+
+def test_frob_partials_of_row_blocks_add_up(lib, torch):
+    """Rows split into uneven blocks (as across GPUs): the blocks' sums add up
+    to the whole matrix's, and the error formed from them matches the oracle's
+    error of the whole matrix."""
+    O, I = 1000, 1152
+    a = syn.host_normal((O, I), 0.02, 4, "A", dtype="bf16")
+    b = syn.as_dtype_values(a + syn.host_normal((O, I), 0.005, 4, "B"), "bf16")
+    A, B = dev(a, "bf16"), dev(b, "bf16")
+    ws = torch.empty(lib.theta_workspace_size(lib.THETA_OP_FROB_ERROR, 1, 1, 1, 0, 0), dtype=torch.uint8,
+                     device="cuda")
+    whole = torch.empty(2, dtype=torch.float64, device="cuda")
+    lib.theta_frob_partials(A, B, whole, ws)
+    tot = torch.zeros(2, dtype=torch.float64, device="cuda")
+    for o0, o1 in ((0, 336), (336, 672), (672, 1000)):
+        part = torch.empty(2, dtype=torch.float64, device="cuda")
+        lib.theta_frob_partials(A[o0:o1], B[o0:o1], part, ws)
+        tot += part
+    w, t = whole.cpu().tolist(), tot.cpu().tolist()
+    assert abs(w[0] - t[0]) <= 1e-12 * w[0] and abs(w[1] - t[1]) <= 1e-12 * w[1]
+    assert_scalar_close(oracle.frob_from_partials(*t), oracle.frob_error(a, b), 1e-5, "frob from blocks")
