@@ -102,6 +102,18 @@ __device__ __forceinline__ R ld_stream(const R* p) {
   return __ldg(p);
 }
 
+// One element of the residual w - s*w0 as one fused multiply-add, rounded
+// once to fp32. Stored as bf16 it is rounded a second time; the two roundings
+// agree with one rounding of the exact value except when the fp32 result
+// lands exactly halfway between two bf16 values (every such point is an fp32
+// number, so the first rounding can reach one but never cross it), where the
+// stored value may be the other neighbour: at most one bf16 ulp from the
+// correctly rounded residual.
+template <typename T>
+__device__ __forceinline__ float residual_elem(float s, float w0, float w) {
+  return fmaf(-s, w0, w);
+}
+
 // x / n rounded once (IEEE division). For n a power of two the quotient is
 // x * 2^-k, which is what the multiplication below computes and rounds
 // identically, so the costly division sequence runs only for other n.

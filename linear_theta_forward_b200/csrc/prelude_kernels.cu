@@ -258,7 +258,7 @@ prelude_pipe_kernel(const __grid_constant__ PreludeArgs a) {
             unpack(wl[v], fw);
             unpack(w0[q], f0);
 #pragma unroll
-            for (int e = 0; e < V::N; ++e) rr[e] = fmaf(-sl, f0[e], fw[e]);
+            for (int e = 0; e < V::N; ++e) rr[e] = residual_elem<T>(sl, f0[e], fw[e]);
             rrow[v] = pack(rr, (R*)nullptr);
           }
         }
@@ -473,7 +473,7 @@ prelude_band2_kernel(const __grid_constant__ PreludeArgs a) {
               unpack(wl[v], fw);
               unpack(w0[q], f0);
 #pragma unroll
-              for (int e = 0; e < V::N; ++e) rr[e] = fmaf(-sl, f0[e], fw[e]);
+              for (int e = 0; e < V::N; ++e) rr[e] = residual_elem<T>(sl, f0[e], fw[e]);
               __stcs(rrow + v, pack(rr, (R*)nullptr));  // written once, not read here again
             }
           }

@@ -80,7 +80,7 @@ band_mean_kernel(PtrTable src, int n, int64_t nvec, int64_t count, T* __restrict
 // live in registers (VPT 16-byte vectors per thread). For every layer of the
 // band: two fp32 dot products with identical operation order, a group
 // reduction (warp shuffle, then shared memory across the group's warps),
-// s = <w,W0> / <W0,W0>, then R = fmaf(-s, W0, w) from the registers.
+// s = <w,W0> / <W0,W0>, then R = w - s W0 (residual_elem) from the registers.
 template <typename T, int TPR, int VPT>
 __global__ void __launch_bounds__(kThreads)
 rowscale_band_kernel(const T* __restrict__ W0, PtrTable w, MutPtrTable s_out, MutPtrTable r_out,
@@ -156,7 +156,7 @@ rowscale_band_kernel(const T* __restrict__ W0, PtrTable w, MutPtrTable s_out, Mu
             unpack(b[j], fw);
             unpack(a[j], f0);
 #pragma unroll
-            for (int e = 0; e < V::N; ++e) r[e] = fmaf(-s, f0[e], fw[e]);
+            for (int e = 0; e < V::N; ++e) r[e] = residual_elem<T>(s, f0[e], fw[e]);
             rrow[v] = pack(r, (R*)nullptr);
           }
         }
@@ -190,7 +190,7 @@ rowscale_band_scalar_kernel(const T* __restrict__ W0, PtrTable w, MutPtrTable s_
       if (lane == 0) static_cast<float*>(s_out.p[l])[o] = s;
       if (write_r) {
         T* rl = static_cast<T*>(r_out.p[l]) + o * I;
-        for (int64_t i = lane; i < I; i += 32) rl[i] = from_f32<T>(fmaf(-s, to_f32(w0[i]), to_f32(wl[i])));
+        for (int64_t i = lane; i < I; i += 32) rl[i] = from_f32<T>(residual_elem<T>(s, to_f32(w0[i]), to_f32(wl[i])));
       }
     }
   }
@@ -211,7 +211,7 @@ residual_vec_kernel(const T* __restrict__ w, const T* __restrict__ W0, const flo
     unpack(ld_stream(reinterpret_cast<const Rw*>(w) + v), fw);
     unpack(ld_stream(reinterpret_cast<const Rw*>(W0) + v), f0);
 #pragma unroll
-    for (int e = 0; e < V::N; ++e) r[e] = fmaf(-sc, f0[e], fw[e]);
+    for (int e = 0; e < V::N; ++e) r[e] = residual_elem<T>(sc, f0[e], fw[e]);
     reinterpret_cast<Rw*>(R)[v] = pack(r, (Rw*)nullptr);
   }
 }
@@ -223,7 +223,7 @@ residual_scalar_kernel(const T* __restrict__ w, const T* __restrict__ W0, const 
   pdl_enter(w, W0, s);
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += stride)
-    R[i] = from_f32<T>(fmaf(-s[i / I], to_f32(W0[i]), to_f32(w[i])));
+    R[i] = from_f32<T>(residual_elem<T>(s[i / I], to_f32(W0[i]), to_f32(w[i])));
 }
 
 // ------------------------------------------------------- frobenius error

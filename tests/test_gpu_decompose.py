@@ -6,7 +6,7 @@ import pytest
 
 import oracle
 import synthetic as syn
-from gpu_helpers import assert_close, assert_scalar_close, dev, host, TOL
+from gpu_helpers import assert_close, assert_close_chain, assert_residual_step, assert_scalar_close, dev, host, TOL
 
 pytestmark = pytest.mark.gpu
 
@@ -74,6 +74,7 @@ def test_residual(lib, torch, dt, I):
     R = torch.empty_like(dev(w[0], dt))
     lib.theta_residual(dev(w[0], dt), dev(W0, dt), dev(s, "f32"), R)
     assert_close(host(R), oracle.residual(w[0], W0, s, dt), dt, "R")
+    assert_residual_step(host(R), w[0], W0, s, dt, "R")
 
 
 def test_zero_w0_row_gives_zero_scale(lib, torch):
@@ -100,11 +101,16 @@ def test_zero_w0_row_gives_zero_scale(lib, torch):
                                         ("bf16", 8, 2, 33, 5376),     # one-pass prelude, 4-layer bands
                                         ("bf16", 2, 2, 20, 21504),    # one-pass prelude, widest rows
                                         ("f32", 3, 1, 21, 1000),
-                                        # two-pass prelude (bands of more than 4 layers)
+                                        # bands of more than 4 layers: two-pass prelude, else
+                                        # band mean + row pass
                                         ("f32", 9, 2, 19, 1000),
                                         ("bf16", 60, 1, 3, 5376),
                                         ("bf16", 11, 2, 130, 1152),
-                                        ("bf16", 12, 1, 5, 21504)])  # rows too long: band mean + row pass
+                                        ("bf16", 12, 1, 5, 21504),     # rows too long: band mean + row pass
+                                        ("f32", 30, 1, 7, 5376),
+                                        ("bf16", 26, 1, 40, 6912),     # the 1B down projection at G = 1
+                                        ("bf16", 60, 4, 261, 5376),    # ragged 15-layer bands
+                                        ("bf16", 60, 1, 300, 5376)])   # 60-layer band, many rows
 def test_decompose_prelude(lib, torch, dt, L, G, O, I):
     w = weights(L, O, I, dt, seed=L * G)
     ws = [dev(w[i], dt) for i in range(L)]
@@ -122,7 +128,9 @@ def test_decompose_prelude(lib, torch, dt, L, G, O, I):
         w0_gpu = host(W0[b])
         assert_close(host(s[layer]), oracle.row_scale(w[layer], w0_gpu), "f32", f"s[{layer}]")
         assert_close(host(s[layer]), ref["s"][layer], "f32", f"s[{layer}] (chain)")
-        assert_close(host(R[layer]), ref["R"][layer], dt, f"R[{layer}]")
+        # R: the step on the GPU's own W0 and s exactly, the chain within one ulp
+        assert_residual_step(host(R[layer]), w[layer], w0_gpu, host(s[layer]), dt, f"R[{layer}]")
+        assert_close_chain(host(R[layer]), ref["R"][layer], dt, f"R[{layer}] (chain)")
 
 
 @pytest.mark.parametrize("dt", DTYPES)
@@ -136,6 +144,40 @@ def test_prelude_without_residual(lib, torch, dt):
     ref = oracle.decompose_family(w, G, 0, dt)
     for layer in range(L):
         assert_close(host(s[layer]), ref["s"][layer], "f32", "s")
+
+
+@pytest.mark.parametrize("dt,L,O,I", [("bf16", 26, 40, 6912), ("f32", 30, 9, 5376)])
+def test_long_band_prelude_without_residual(lib, torch, dt, L, O, I):
+    w = weights(L, O, I, dt, seed=7)
+    ws = [dev(w[i], dt) for i in range(L)]
+    W0 = [torch.empty_like(ws[0])]
+    s = [torch.empty(O, dtype=torch.float32, device="cuda") for _ in range(L)]
+    lib.theta_decompose_prelude(ws, 1, W0, s, None)
+    ref = oracle.decompose_family(w, 1, 0, dt)
+    assert_close(host(W0[0]), ref["W0"][0], dt, "W0")
+    for layer in range(L):
+        assert_close(host(s[layer]), ref["s"][layer], "f32", f"s[{layer}]")
+
+
+@pytest.mark.parametrize("dt,L,I", [("bf16", 60, 5376), ("bf16", 26, 6912), ("bf16", 12, 21504)])
+def test_identical_layers_give_exact_scale_in_a_long_band(lib, torch, dt, L, I):
+    """Every layer of a long band equal (bf16 weights; two-pass and band mean +
+    row pass routes): the mean is that weight exactly -- up to 256 copies of
+    an 8-bit significand sum exactly in fp32 -- and the two dot products of
+    each row use one operation order, so s == 1 and the residual is 0 bit for
+    bit. (fp32 weights have no such guarantee: k copies of a 24-bit
+    significand already round at k = 3.)"""
+    O = 24
+    one = weights(1, O, I, dt, seed=9)[0]
+    ws = [dev(one, dt) for _ in range(L)]
+    W0 = [torch.empty_like(ws[0])]
+    s = [torch.empty(O, dtype=torch.float32, device="cuda") for _ in range(L)]
+    R = [torch.full_like(ws[0], 7.0) for _ in range(L)]
+    lib.theta_decompose_prelude(ws, 1, W0, s, R)
+    assert torch.equal(W0[0], ws[0])
+    for layer in range(L):
+        assert bool((s[layer] == 1.0).all()), layer
+        assert bool((R[layer] == 0).all()), layer
 
 
 @pytest.mark.parametrize("dt", DTYPES)
