@@ -21,7 +21,7 @@ N(0,0.01), activations X ~ N(0,1)):
 
 The stages are (entry points of libtheta):
   prelude      theta_decompose_prelude      W0 per band, s and R per layer
-  reconstruct  theta_reconstruct            diag(s).W0 + U.V^T per layer
+  reconstruct  theta_reconstruct_band       diag(s).W0 + U.V^T for the layers of a band
   frob         theta_frob_error             ||W - W_rec||_F / ||W||_F per layer
   forward      theta_linear_forward (one or two tokens on Gemma-3-1B shapes:
                theta_linear_forward_grouped, one call for all 182 problems)
@@ -144,6 +144,16 @@ def prelude_launches(L, G, I, b=BF16, num_sms=148):
     return G + 1
 
 
+def reconstruct_band_launches(L, G, r):
+    """Kernel launches of the theta_reconstruct_band calls of one family, one
+    call per band: one launch per 64 layers of a band, or one per layer for
+    one-layer bands, rank 0 or rank above 128."""
+    sizes = [L // G + (1 if b < L % G else 0) for b in range(G)]
+    if r == 0 or r > 128:
+        return L
+    return sum(1 if n == 1 else -(-n // 64) for n in sizes)
+
+
 def grouped_stage(cfg, M):
     """One or two tokens on Gemma-3-1B shapes: one grouped call per stage."""
     return M <= 2 and cfg.model.name == syn.GEMMA3_1B.name
@@ -178,8 +188,8 @@ def plan_stages(cfg: Config, grouped=True):
             # the layers of a band read one W0: once per band from HBM
             u = b - (L - G) * sum(O * I * BF16 for (O, I) in fams.values())
             out.append(dict(cfg=cfg.key, kind="reconstruct", G=G, M=0, bytes=b, unique=u,
-                            flops=L * sum(2 * O * I * r for (O, I) in fams.values()), calls=nf * L,
-                            launches=nf * L))
+                            flops=L * sum(2 * O * I * r for (O, I) in fams.values()), calls=nf * G,
+                            launches=nf * reconstruct_band_launches(L, G, r)))
             b = L * sum(bytes_frob(O, I) for (O, I) in fams.values())
             out.append(dict(cfg=cfg.key, kind="frob", G=G, M=0, bytes=b, unique=b, flops=0, calls=nf * L,
                             launches=2 * nf * L))
@@ -537,10 +547,15 @@ class Workload:
                                           for f in fams])
         band = d["bands"][G]
         if st["kind"] == "reconstruct":
-            return lambda: self._fan_out([lambda s, f=f, l=l: t.theta_reconstruct(d["s"][f][l], d["W0"][f][band[l]],
-                                                                                 d["U"][f][l], d["V"][f][l],
-                                                                                 d["rec"][f][l])
-                                          for l in range(L) for f in fams])
+            # one call per band: each W0 tile read once for all the band's layers
+            calls = []
+            for f in fams:
+                for b in range(G):
+                    ls = [l for l in range(L) if band[l] == b]
+                    calls.append(lambda s, f=f, b=b, ls=ls: t.theta_reconstruct_band(
+                        [d["s"][f][l] for l in ls], d["W0"][f][b], [d["U"][f][l] for l in ls],
+                        [d["V"][f][l] for l in ls], [d["rec"][f][l] for l in ls]))
+            return lambda: self._fan_out(calls)
         if st["kind"] == "frob":
             gi = cfg.G.index(G)
             fi = {f: i for i, f in enumerate(fams)}

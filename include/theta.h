@@ -193,6 +193,23 @@ int theta_reconstruct(const float* s, const void* W0, const void* U, const void*
                       int64_t I, int rank, theta_dtype dt, void* W_out, void* stream);
 
 /*
+ * theta_reconstruct_band -- theta_reconstruct for the n layers of one band,
+ * which share one W0 ("Banded sharing"; "The theta bundle" -- the
+ * approximation formula): W_out[l] = diag(s[l]) . W0 + U[l] . V[l]^T.
+ *
+ *   s, U, V, W_out  host arrays of n device pointers (one per layer), each as
+ *                   in theta_reconstruct; U and V may be NULL when rank == 0.
+ *   W0       device [O, I], the band's shared block.
+ *   1 <= n <= THETA_MAX_LAYERS; other rules as theta_reconstruct.
+ * Every output is element for element what theta_reconstruct gives for that
+ * layer; the bf16 path reads each 128 x 128 tile of W0 once for all the
+ * layers (up to 64 layers per launch, rank <= 128; otherwise one
+ * theta_reconstruct per layer), fp32 runs theta_reconstruct per layer.
+ */
+int theta_reconstruct_band(const float* const* s, const void* W0, const void* const* U, const void* const* V, int n,
+                           int64_t O, int64_t I, int rank, theta_dtype dt, void* const* W_out, void* stream);
+
+/*
  * theta_frob_error -- relative_frobenius_error(original, reconstructed)
  * = ||A - B||_F / ||A||_F ("Quality" -- Reconstruction error; "The theta
  * bundle" -- relative_frobenius_error). 0 if both norms are 0, +inf if only

@@ -21,7 +21,7 @@ __all__ = [
     "theta_forward_problem", "ForwardGroup", "theta_linear_forward_grouped",
     "theta_version", "theta_status_string", "theta_last_error", "theta_band_index",
     "theta_band_mean", "theta_row_scale", "theta_residual", "theta_decompose_prelude",
-    "theta_reconstruct", "theta_frob_error", "theta_frob_partials", "theta_linear_forward", "theta_workspace_size",
+    "theta_reconstruct", "theta_reconstruct_band", "theta_frob_error", "theta_frob_partials", "theta_linear_forward", "theta_workspace_size",
     "theta_device_status", "theta_linear_forward_noalloc", "theta_set_policy", "theta_get_policy",
     "theta_selftest_wait_timeout", "THETA_POLICY_LATENCY", "THETA_POLICY_THROUGHPUT",
 ]
@@ -56,6 +56,7 @@ _SIGNATURES = {
     "theta_reconstruct": (_int, _vp, _vp, _vp, _vp, _i64, _i64, _int, _int, _vp, _vp),
     "theta_frob_error": (_int, _vp, _vp, _i64, _int, _vp, _vp, _sz, _vp),
     "theta_frob_partials": (_int, _vp, _vp, _i64, _int, _vp, _vp, _sz, _vp),
+    "theta_reconstruct_band": (_int, _vp, _vp, _vp, _vp, _int, _i64, _i64, _int, _int, _vp, _vp),
     "theta_linear_forward": (_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp, _sz, _vp),
     "theta_linear_forward_noalloc": (_int, _vp, _i64, _i64, _vp, _i64, _vp, _vp, _vp, _int, _int, _vp, _vp),
     "theta_nvfp4_quantize": (_int, _vp, _i64, _i64, _vp, _vp, _vp, _vp, _sz, _vp),
@@ -221,6 +222,22 @@ def theta_reconstruct(s, W0, U, V, W_out, stream=None) -> None:
     _check(_load().theta_reconstruct(_ptr(s, "s"), _ptr(W0, "W0"), _ptr(U, "U", optional=True),
                                  _ptr(V, "V", optional=True), O, I, rank, _dtype_code(W0),
                                  _ptr(W_out, "W_out"), _stream(stream)), "theta_reconstruct")
+
+
+def theta_reconstruct_band(s, W0, U, V, W_out, stream=None) -> None:
+    """The reconstructions of the layers of one band: s, U, V, W_out are
+    lists with one tensor per layer (U and V None for rank 0); W0 is shared."""
+    O, I = W0.shape
+    rank = 0 if U is None else U[0].shape[1]
+    sp = _ptr_array(s, "s")
+    op = _ptr_array(W_out, "W_out")
+    up = _ptr_array(U, "U") if rank > 0 else None
+    vp = _ptr_array(V, "V") if rank > 0 else None
+    _check(_load().theta_reconstruct_band(ctypes.cast(sp, _vp), _ptr(W0, "W0"),
+                                      ctypes.cast(up, _vp) if up is not None else None,
+                                      ctypes.cast(vp, _vp) if vp is not None else None, len(s), O, I, rank,
+                                      _dtype_code(W0), ctypes.cast(op, _vp), _stream(stream)),
+           "theta_reconstruct_band")
 
 
 def theta_frob_error(original, reconstructed, out, workspace, stream=None) -> None:

@@ -112,5 +112,10 @@ int launch_gate_up_umma(const LaunchCtx& c, const void* X, const void* W0g, cons
 int launch_reconstruct_umma(const LaunchCtx& c, const float* s, const void* W0, const void* U,
                             const void* V, int64_t O, int64_t I, int r, void* W_out,
                             cudaError_t* cuda_err);
+// The n layers of one band (one shared W0): each W0 tile read once for all of
+// them (bands of up to 64 layers per launch; rank <= 128; else per layer).
+int launch_reconstruct_band_umma(const LaunchCtx& c, const float* const* s, const void* W0, const void* const* U,
+                                 const void* const* V, int n, int64_t O, int64_t I, int r, void* const* W_out,
+                                 cudaError_t* cuda_err);
 
 }  // namespace theta

@@ -273,6 +273,47 @@ THETA_API int theta_reconstruct(const float* s, const void* W0, const void* U, c
   return THETA_OK;
 }
 
+THETA_API int theta_reconstruct_band(const float* const* s, const void* W0, const void* const* U,
+                                     const void* const* V, int n, int64_t O, int64_t I, int rank, theta_dtype dt,
+                                     void* const* W_out, void* stream) {
+  if (!valid_dt(dt)) return fail(THETA_ERR_INVALID_ARG, "theta_reconstruct_band: bad dtype %d", (int)dt);
+  if (n < 1 || n > THETA_MAX_LAYERS)
+    return fail(THETA_ERR_INVALID_ARG, "theta_reconstruct_band: n=%d outside [1, %d]", n, THETA_MAX_LAYERS);
+  if (O < 1 || I < 1 || rank < 0)
+    return fail(THETA_ERR_INVALID_ARG, "theta_reconstruct_band: need O, I >= 1 and rank >= 0");
+  if (!s || !W0 || !W_out || (rank > 0 && (!U || !V)))
+    return fail(THETA_ERR_INVALID_ARG, "theta_reconstruct_band: NULL array");
+  for (int l = 0; l < n; ++l)
+    if (!s[l] || !W_out[l] || (rank > 0 && (!U[l] || !V[l])))
+      return fail(THETA_ERR_INVALID_ARG, "theta_reconstruct_band: NULL pointer for layer %d", l);
+  if (dt == THETA_BF16) {
+    bool ok = aligned16(W0) && I % 8 == 0 && rank % 8 == 0;
+    for (int l = 0; l < n && ok; ++l)
+      ok = aligned16(s[l]) && aligned16(W_out[l]) && (rank == 0 || (aligned16(U[l]) && aligned16(V[l])));
+    if (!ok)
+      return fail(THETA_ERR_ALIGNMENT,
+                  "theta_reconstruct_band: bf16 needs 16-byte aligned pointers and I, rank multiples of 8");
+  } else if (O > kSimtMaxRows) {
+    return fail(THETA_ERR_UNSUPPORTED, "theta_reconstruct_band: fp32 path takes at most %lld rows",
+                (long long)kSimtMaxRows);
+  }
+  LaunchCtx c;
+  int st = make_ctx(stream, &c);
+  if (st) return st;
+  if (dt == THETA_BF16) {
+    cudaError_t ce = cudaSuccess;
+    st = launch_reconstruct_band_umma(c, s, W0, rank > 0 ? U : nullptr, rank > 0 ? V : nullptr, n, O, I, rank,
+                                      W_out, &ce);
+    if (st == THETA_ERR_CUDA) return fail_cuda(ce, "theta_reconstruct_band (tensor-core path)");
+    return st;
+  }
+  for (int l = 0; l < n; ++l)
+    CHECK_LAUNCH(launch_reconstruct_simt(c, dt, s[l], W0, rank > 0 ? U[l] : nullptr, rank > 0 ? V[l] : nullptr, O,
+                                         I, rank, W_out[l]),
+                 "theta_reconstruct_band launch");
+  return THETA_OK;
+}
+
 THETA_API int theta_frob_error(const void* original, const void* reconstructed, int64_t n,
                                theta_dtype dt, double* out, void* workspace,
                                size_t workspace_bytes, void* stream) {

@@ -536,6 +536,213 @@ recon_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
   if (warp == 1) ptx::tmem_dealloc(tmem, kRecN);
 }
 
+// --------------------------------------------------------- band reconstruct
+// The reconstructions of the n layers of one band, which share W0:
+// W_l = diag(s_l).W0 + U_l.V_l^T for l < n. One CTA per 128 x 128 tile of W0
+// loads that tile once and loops over the layers:
+//   warp 0    TMA: the W0 tile, then layer by layer the U_l and V_l rank
+//             blocks into a double buffer
+//   warp 1    the K = rank MMAs of layer l into one of two tensor-memory
+//             accumulators, once the epilogue has read layer l-2's product
+//             from it
+//   warps 2-9 the epilogue, two warps per 32-lane quarter of tensor memory
+//             (64 columns each): U_l.V_l^T from tensor memory plus s_l * W0
+//             from the tile, rounded to bf16 into one of several output tiles
+//             that one thread stores by TMA, several stores in flight
+// So W0 crosses HBM once per band instead of once per layer, and layer l+1's
+// loads and MMAs overlap layer l's epilogue and store. Same arithmetic as
+// recon_kernel, element for element.
+constexpr int kBandMax = 64;  // layers per launch (their tensor maps travel as kernel parameters)
+constexpr int kBandThreads = 320;  // producer, MMA issuer, 8 epilogue warps
+constexpr int kBandEpi = 256;      // epilogue threads
+
+struct BandArgs {
+  CUtensorMap U[kBandMax], V[kBandMax], Out[kBandMax];
+  const float* s[kBandMax];
+  int n, O, I;
+  unsigned* err;
+};
+
+template <int KB>
+struct BandCfg {
+  static constexpr int kUBlock = kBM * 128;    // 128 rows x 64 rank columns (bf16)
+  static constexpr int kVBlock = kRecN * 128;
+  static constexpr int kUVBytes = KB * (kUBlock + kVBlock);  // one layer's U and V blocks
+  static constexpr int kTileBytes = (kRecN / kBK) * kABytes;  // a 128 x 128 bf16 tile as two 64-column boxes
+  // output tiles whose stores may be in flight at once (the writes are the
+  // kernel's traffic; each SM needs ~100 KB of them in flight)
+  static constexpr int kOutBufs = KB == 1 ? 4 : 2;
+  static constexpr int kSmemBytes = kTileBytes + 2 * kUVBytes + kOutBufs * kTileBytes + 1024 + 256;
+};
+
+template <int KB>
+__global__ void __launch_bounds__(kBandThreads, 1)
+recon_band_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constant__ BandArgs a) {
+  using C = BandCfg<KB>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sW = smem;
+  uint8_t* sUV = sW + C::kTileBytes;                 // [2][U blocks, V blocks]
+  uint8_t* sOut = sUV + 2 * C::kUVBytes;             // [kOutBufs] output tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOut + C::kOutBufs * C::kTileBytes);
+  uint64_t* w_full = bars;            // the W0 tile landed
+  uint64_t* uv_full = bars + 1;       // [2] a layer's U, V blocks landed
+  uint64_t* uv_empty = bars + 3;      // [2] the MMAs reading them are done
+  uint64_t* acc_full = bars + 5;      // [2] a layer's product in tensor memory
+  uint64_t* acc_free = bars + 7;      // [2] the epilogue has read it
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 9);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int i0 = blockIdx.x * kRecN, o0 = blockIdx.y * kBM;
+  const int n = a.n;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(w_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&uv_full[b], 1);
+      ptx::mbar_init(&uv_empty[b], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&acc_full[b], 1);
+      ptx::mbar_init(&acc_free[b], kBandEpi);
+    }
+    *abort_flag = prior_timeout(a.err);
+    ptx::fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, 2 * kRecN);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_enter();
+
+  auto give_up = [&]() {
+    record_timeout(a.err);
+    *abort_flag = 1;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      ptx::mbar_arrive_expect_tx(w_full, C::kTileBytes);
+#pragma unroll
+      for (int bx = 0; bx < kRecN / kBK; ++bx) ptx::tma_load_2d(sW + bx * kABytes, &tmW0, w_full, i0 + bx * kBK, o0);
+      int issued = 0;
+      for (int l = 0; l < n; ++l) {
+        const int b = l & 1;
+        if (l >= 2 && !ptx::mbar_wait(&uv_empty[b], (uint32_t)(((l - 2) >> 1) & 1), abort_flag)) {
+          give_up();
+          break;
+        }
+        uint8_t* u = sUV + b * C::kUVBytes;
+        uint8_t* v = u + KB * C::kUBlock;
+        ptx::mbar_arrive_expect_tx(&uv_full[b], C::kUVBytes);
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb) {
+          ptx::tma_load_2d(u + kb * C::kUBlock, &a.U[l], &uv_full[b], kb * kBK, o0);
+          ptx::tma_load_2d(v + kb * C::kVBlock, &a.V[l], &uv_full[b], kb * kBK, i0);
+        }
+        ++issued;
+      }
+      // every load lands before the CTA can leave (immediate unless aborted)
+      int never = 0;
+      ptx::mbar_wait(w_full, 0, &never);
+      for (int b = 0; b < 2 && b < issued; ++b) {
+        const int last = b + ((issued - 1 - b) / 2) * 2;
+        ptx::mbar_wait(&uv_full[b], (uint32_t)((last >> 1) & 1), &never);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = ptx::idesc_bf16(kBM, kRecN, 0);
+      int done = 0;
+      for (int l = 0; l < n; ++l) {
+        const int b = l & 1;
+        // buffer b of tensor memory was last read by the epilogue of layer l-2
+        if (!ptx::mbar_wait(&uv_full[b], (uint32_t)((l >> 1) & 1), abort_flag) ||
+            (l >= 2 && !ptx::mbar_wait(&acc_free[b], (uint32_t)(((l - 2) >> 1) & 1), abort_flag))) {
+          give_up();
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t ua = ptx::smem_u32(sUV + b * C::kUVBytes), va = ua + KB * C::kUBlock;
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            ptx::umma_bf16(tmem + (uint32_t)(b * kRecN), ptx::sdesc_sw128(ua + kb * C::kUBlock + kk * 32, 16, 1024),
+                           ptx::sdesc_sw128(va + kb * C::kVBlock + kk * 32, 16, 1024), idesc, (kb | kk) ? 1u : 0u);
+        ptx::umma_commit(&acc_full[b]);
+        ptx::umma_commit(&uv_empty[b]);
+        ++done;
+      }
+      if (done < n && done > 0) {
+        // aborted: the issued MMAs finish before tensor memory is freed
+        int never = 0;
+        const int last = done - 1;
+        ptx::mbar_wait(&acc_full[last & 1], (uint32_t)((last >> 1) & 1), &never);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;         // a warp reads lanes 32 * (warp % 4) ...
+    const int half = (warp - 2) / 4;      // ... and columns 64 * half ... + 63
+    const int row = quarter * 32 + lane;  // tensor-memory lane = row of the tile
+    const uint32_t taddr0 = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * 64);
+    const bool leader = threadIdx.x == 64;  // issues the stores
+    bool ok = ptx::mbar_wait(w_full, 0, abort_flag);
+    for (int l = 0; l < n && ok; ++l) {
+      const int b = l & 1;
+      const uint32_t taddr = taddr0 + (uint32_t)(b * kRecN);
+      ok = ptx::mbar_wait(&acc_full[b], (uint32_t)((l >> 1) & 1), abort_flag);
+      // the store of layer l - kOutBufs read its buffer before this layer rewrites it
+      if (leader) ptx::bulk_wait_read_n<C::kOutBufs - 1>();
+      ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld is warp-collective
+      asm volatile("bar.sync 1, %0;" ::"n"(kBandEpi) : "memory");
+      if (!ok) break;
+      ptx::tc_fence_after();
+      const float so = (o0 + row < a.O) ? __ldg(a.s[l] + o0 + row) : 0.f;
+      // this warp's 64 columns (one swizzled box of the tile): all four loads
+      // in flight, one wait
+      float d[64];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) ptx::tmem_ld16(taddr + q * 16, *reinterpret_cast<float(*)[16]>(d + 16 * q));
+      ptx::tmem_wait_ld();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&acc_free[b]);  // tensor memory read: layer l+2's MMAs may start
+      const uint8_t* wbox = sW + half * kABytes + row * 128;
+      uint8_t* obox = sOut + (l % C::kOutBufs) * C::kTileBytes + half * kABytes + row * 128;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int chunk = k ^ (row & 7);  // 128-byte swizzle of 16-byte chunks
+        float w[8], o[8];
+        unpack(*reinterpret_cast<const uint4*>(wbox + chunk * 16), w);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) o[e] = fmaf(so, w[e], d[8 * k + e]);
+        *reinterpret_cast<uint4*>(obox + chunk * 16) = pack(o, (uint4*)nullptr);
+      }
+      ptx::fence_proxy_async_smem();
+      asm volatile("bar.sync 1, %0;" ::"n"(kBandEpi) : "memory");
+      if (leader) {
+        const uint8_t* out = sOut + (l % C::kOutBufs) * C::kTileBytes;
+#pragma unroll
+        for (int bx = 0; bx < kRecN / kBK; ++bx)
+          if (i0 + bx * kBK < a.I) ptx::tma_store_2d(&a.Out[l], out + bx * kABytes, i0 + bx * kBK, o0);
+        ptx::bulk_commit();
+      }
+    }
+    if (!ok && !*abort_flag) give_up();
+    if (leader) ptx::bulk_wait_read();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) ptx::tmem_dealloc(tmem, 2 * kRecN);
+}
+
 // ------------------------------------------------------------------ host side
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -698,6 +905,17 @@ cudaError_t launch_recon(const LaunchCtx& c, const CUtensorMap& mU, const CUtens
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3((unsigned)ceil_div(I, kRecN), (unsigned)ceil_div(O, kBM), 1), dim3(kRecThreads),
                     C::kSmemBytes, c.stream, 1, mU, mV, mW0, mOut, s, O, I, c.err);
+}
+
+template <int KB>
+cudaError_t launch_band(const LaunchCtx& c, const CUtensorMap& mW0, const BandArgs& a) {
+  using C = BandCfg<KB>;
+  auto kern = recon_band_kernel<KB>;
+  static KernelInfo info[64];
+  cudaError_t e = prepare_kernel(&info[c.device], c.device, kern, kBandThreads, C::kSmemBytes, 2 * kRecN, false);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3((unsigned)ceil_div(a.I, kRecN), (unsigned)ceil_div(a.O, kBM), 1), dim3(kBandThreads),
+                    C::kSmemBytes, c.stream, 1, mW0, a);
 }
 
 // The failure path of every bounded wait, on purpose: one thread waits on an
@@ -889,6 +1107,45 @@ int launch_gate_up_umma(const LaunchCtx& c, const void* X, const void* W0g, cons
   if (e != cudaSuccess) {
     *ce = e;
     return THETA_ERR_CUDA;
+  }
+  return THETA_OK;
+}
+
+int launch_reconstruct_band_umma(const LaunchCtx& c, const float* const* s, const void* W0, const void* const* U,
+                                 const void* const* V, int n, int64_t O, int64_t I, int r, void* const* W_out,
+                                 cudaError_t* ce) {
+  *ce = cudaSuccess;
+  // one layer, rank 0 or a rank beyond two 64-column blocks: one call per layer
+  if (n == 1 || r == 0 || r > 2 * kBK) {
+    for (int l = 0; l < n; ++l) {
+      const int st = launch_reconstruct_umma(c, s[l], W0, r > 0 ? U[l] : nullptr, r > 0 ? V[l] : nullptr, O, I, r,
+                                             W_out[l], ce);
+      if (st) return st;
+    }
+    return THETA_OK;
+  }
+  if (O > (int64_t)65535 * kBM || I > ((int64_t)1 << 31) - 256) return THETA_ERR_UNSUPPORTED;
+  static thread_local BandArgs a;  // ~25 KB of tensor maps: kept off the stack
+  CUtensorMap mW0;
+  int st;
+  if ((st = make_map(&mW0, W0, O, I, kBM, ce))) return st;
+  for (int l0 = 0; l0 < n; l0 += kBandMax) {
+    const int m = n - l0 < kBandMax ? n - l0 : kBandMax;
+    for (int j = 0; j < m; ++j) {
+      if ((st = make_map(&a.U[j], U[l0 + j], O, r, kBM, ce))) return st;
+      if ((st = make_map(&a.V[j], V[l0 + j], I, r, kRecN, ce))) return st;
+      if ((st = make_map(&a.Out[j], W_out[l0 + j], O, I, kBM, ce))) return st;
+      a.s[j] = s[l0 + j];
+    }
+    a.n = m;
+    a.O = (int)O;
+    a.I = (int)I;
+    a.err = c.err;
+    const cudaError_t e = r > kBK ? launch_band<2>(c, mW0, a) : launch_band<1>(c, mW0, a);
+    if (e != cudaSuccess) {
+      *ce = e;
+      return THETA_ERR_CUDA;
+    }
   }
   return THETA_OK;
 }

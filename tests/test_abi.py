@@ -116,6 +116,20 @@ def test_sizes_beyond_the_grid_limits_are_refused_on_the_host(lib):
     assert raw.theta_reconstruct(p, p, None, None, M32, 64, 0, 0, p, None) == -2
 
 
+def test_reconstruct_band_validation(lib):
+    raw = lib.lib
+    p = ctypes.c_void_p(16)
+    arr = (ctypes.c_void_p * 2)(16, 16)
+    bad = (ctypes.c_void_p * 2)(16, None)
+    a = ctypes.cast(arr, ctypes.c_void_p)
+    assert raw.theta_reconstruct_band(a, p, a, a, 0, 8, 8, 8, 1, a, None) == -1            # n = 0
+    assert raw.theta_reconstruct_band(a, p, a, a, 300, 8, 8, 8, 1, a, None) == -1          # n > max
+    assert raw.theta_reconstruct_band(None, p, a, a, 2, 8, 8, 8, 1, a, None) == -1         # NULL array
+    assert raw.theta_reconstruct_band(a, p, ctypes.cast(bad, ctypes.c_void_p), a, 2, 8, 8, 8, 1, a, None) == -1
+    assert raw.theta_reconstruct_band(a, p, a, a, 2, 8, 12, 8, 1, a, None) == -3           # I % 8
+    assert raw.theta_reconstruct_band(a, p, a, a, 2, 8, 8, 8, 7, a, None) == -1            # dtype
+
+
 def test_nvfp4_validation(lib):
     raw = lib.lib
     p = ctypes.c_void_p(16)

@@ -45,8 +45,14 @@ def test_launch_counts_per_step():
     pre = {s["name"]: s["launches"] for s in grouped if s["kind"] == "prelude"}
     assert pre == {"C1.prelude.G26": 7, "C1.prelude.G1": 7, "C4.prelude.G1": 2, "C4.prelude.G4": 1,
                    "C4.prelude.G15": 1, "C4.prelude.G60": 1}
-    assert sum(s["launches"] for s in grouped) == 12315
-    assert sum(s["launches"] for s in per_call) == 12315 + 4 * (364 - 3)
+    # reconstruct: one band call per (family, band); a one-layer band is one
+    # per-layer launch (C1 at G = 26: 182; G = 1: 7; C4: 1 + 4 + 15 + 60)
+    rec = {s["name"]: s["launches"] for s in grouped if s["kind"] == "reconstruct"}
+    assert rec == {"C1.reconstruct.G26": 182, "C1.reconstruct.G1": 7, "C4.reconstruct.G1": 1,
+                   "C4.reconstruct.G4": 4, "C4.reconstruct.G15": 15, "C4.reconstruct.G60": 60}
+    assert bench.reconstruct_band_launches(130, 1, 64) == 3 and bench.reconstruct_band_launches(10, 2, 0) == 10
+    assert sum(s["launches"] for s in grouped) == 11980
+    assert sum(s["launches"] for s in per_call) == 11980 + 4 * (364 - 3)
 
 
 @pytest.mark.parametrize("key", ["C1", "C2", "C3", "C4"])

@@ -146,6 +146,36 @@ def test_reconstruct(lib, torch, dt, O, I, r):
     assert_close(host(out), oracle.reconstruct(s, W0, U, V, dt), dt, "W_rec")
 
 
+BAND_CASES = [("bf16", 4, 256, 264, 16), ("bf16", 7, 300, 1152, 32), ("bf16", 15, 1024, 5376, 64),
+              ("bf16", 3, 130, 200, 128), ("bf16", 70, 64, 256, 8), ("bf16", 2, 40, 64, 0),
+              ("bf16", 5, 2056, 136, 64), ("f32", 3, 72, 96, 16)]
+
+
+@pytest.mark.parametrize("dt,n,O,I,r", BAND_CASES)
+def test_reconstruct_band(lib, torch, dt, n, O, I, r):
+    """theta_reconstruct_band over the n layers of one band: each output
+    equals theta_reconstruct of that layer element for element, and the
+    oracle's reconstruct within the tolerance (bands of more than 64 layers
+    take two launches; rank 0 and fp32 take one call per layer)."""
+    W0 = syn.host_normal((O, I), 0.02, n + O, "W0-band", dtype=dt)
+    s = [1.0 + syn.host_normal((O,), 0.05, n + O, "s-band", l) for l in range(n)]
+    U = [syn.host_normal((O, r), 0.05, n + O, "U-band", l, dtype=dt) for l in range(n)]
+    V = [syn.host_normal((I, r), 0.05, n + O, "V-band", l, dtype=dt) for l in range(n)]
+    d_s = [dev(x, "f32") for x in s]
+    d_U = [dev(x, dt) for x in U] if r else None
+    d_V = [dev(x, dt) for x in V] if r else None
+    d_W0 = dev(W0, dt)
+    outs = [torch.full((O, I), float("nan"), dtype=d_W0.dtype, device="cuda") for _ in range(n)]
+    lib.theta_reconstruct_band(d_s, d_W0, d_U, d_V, outs)
+    one = torch.empty_like(outs[0])
+    for l in range(n):
+        lib.theta_reconstruct(d_s[l], d_W0, d_U[l] if r else None, d_V[l] if r else None, one)
+        assert torch.equal(outs[l], one), f"layer {l}: differs from theta_reconstruct"
+        if l in (0, n // 2, n - 1):
+            assert_close(host(outs[l]), oracle.reconstruct(s[l], W0, U[l], V[l], dt), dt, f"W_rec[{l}]")
+    lib.theta_device_status()
+
+
 def test_tiny_workload_end_to_end(lib, torch):
     """The tiny workload: 4 layers [256, 256] fp32, G = 2, rank 8 from the
     oracle's SVD of each residual, X [16, 256]; the GPU runs the prelude,
