@@ -1125,34 +1125,43 @@ def run_op(args):
         call()
     torch.cuda.synchronize()
     theta.theta_device_status()
+    # the sampler starts first (nvidia-smi needs a moment), and the timed
+    # region repeats until it spans at least 0.6 s, so that the clocks seen
+    # while it ran are on record
     with ClockSampler(0, period_ms=20) as clocks:
-        if args.b2b:
-            # calls back to back between one pair of events; only meaningful
-            # for HBM when one call moves well over the 126 MB L2
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record()
-            for _ in range(args.iters):
-                call()
-            b.record()
-            torch.cuda.synchronize()
-            ms = a.elapsed_time(b) / args.iters
-            l2 = "calls back to back, no flush (mean of %d)" % args.iters
-            if args.op in ("forward", "forward_nvfp4", "gate_up"):
-                l2 += ", cycling over %d independent problems" % args.bufs
-        else:
-            times = []
-            for _ in range(args.iters):
-                flush.fill_(1)
+        time.sleep(0.3)
+        t_end = time.perf_counter() + 0.6
+        rounds, per_call = 0, []
+        while rounds == 0 or time.perf_counter() < t_end:
+            if args.b2b:
+                # calls back to back between one pair of events; only meaningful
+                # for HBM when one call moves well over the 126 MB L2
                 a = torch.cuda.Event(enable_timing=True)
                 b = torch.cuda.Event(enable_timing=True)
                 a.record()
-                call()
+                for _ in range(args.iters):
+                    call()
                 b.record()
                 torch.cuda.synchronize()
-                times.append(a.elapsed_time(b))
-            ms = statistics.median(times)
-            l2 = "flushed (256 MiB write) before every call"
+                per_call.append(a.elapsed_time(b) / args.iters)
+            else:
+                for _ in range(args.iters):
+                    flush.fill_(1)
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record()
+                    call()
+                    b.record()
+                    torch.cuda.synchronize()
+                    per_call.append(a.elapsed_time(b))
+            rounds += 1
+    ms = statistics.median(per_call)
+    if args.b2b:
+        l2 = "calls back to back, no flush (median over %d rounds of %d calls)" % (rounds, args.iters)
+        if args.op in ("forward", "forward_nvfp4", "gate_up"):
+            l2 += ", cycling over %d independent problems" % args.bufs
+    else:
+        l2 = "flushed (256 MiB write) before every call (median of %d)" % len(per_call)
     theta.theta_device_status()
     line = {"op": args.op, "shape": {"M": M, "O": O, "I": I, "rank": r, "layers": L, "G": G}, "dtype": "bf16",
             "ms": round(ms, 5), "iters": args.iters, "l2": l2,
