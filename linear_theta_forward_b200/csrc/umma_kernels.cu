@@ -380,6 +380,237 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
   if (warp == 1) ptx::tmem_dealloc(tmem, C::kTmemCols);
 }
 
+// ------------------------------------------------------------ CTA-pair forward
+// The FORWARD epilogue over 256 x 256 tiles (weight rows x tokens) on pairs
+// of SMs: the two CTAs of a cluster of two share each tcgen05 MMA of M = 256,
+// N = 256 (cta_group::2), issued by the even CTA. Each CTA stages its own half
+// of both operands -- 128 weight rows and 128 tokens, 32 KB per 64-wide K
+// block -- and receives its 128 rows x 256 tokens of D1 and D2 in its own
+// tensor memory. Per K block an SM takes in two thirds of what a 128 x 256
+// tile on one SM does for the same tensor work.
+//
+// The kernel is persistent: a cluster walks the tiles c, c + clusters, ...
+// Its producers load the next tile's stages while the epilogue still works
+// on the current one, and the epilogue hands tensor memory back as soon as it
+// has moved the tile into shared memory (s * D1 + D2, rounded to bf16, as
+// [token][row] -- the layout of Y), before one TMA store writes it out. So
+// between two tiles the tensor pipe waits only for that drain, not for a CTA
+// to finish, launch and fill its pipeline.
+//
+// Each CTA's producer signals the even CTA's full barrier (which expects
+// both halves); MMA completion is committed to the empty and accumulator
+// barriers of both CTAs; the epilogue warps of both CTAs arrive on the even
+// CTA's tensor-memory-free barrier.
+constexpr int kPairN = 256;                                     // tokens per pair tile: MMA N
+constexpr int kPairHalf = kPairN / 2;                           // tokens staged by each CTA
+constexpr int kPairStageBytes = kABytes + kPairHalf * kBK * 2;  // 16 KB of W0 (or U) + 16 KB of X (or T)
+constexpr int kPairStages = 5;
+constexpr int kPairOutBytes = kBM * kPairN * 2;                 // a CTA's Y tile, bf16 [token][row]
+constexpr int kPairTmemCols = 2 * kPairN;                       // D1, D2
+constexpr int kPairSmemBytes = kPairStages * kPairStageBytes + kPairOutBytes + 1024 /*align*/ + 256 /*barriers*/;
+constexpr uint16_t kPairMask = 0x3;                             // both CTAs of the cluster
+constexpr int kPairEpi = 128;                                   // epilogue threads per CTA
+
+__global__ void __launch_bounds__(kThreads)
+pair_forward_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+                    const __grid_constant__ CUtensorMap tmB3, const __grid_constant__ CUtensorMap tmY,
+                    const Args args) {
+  constexpr int S = kPairStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  bf16* sOut = reinterpret_cast<bf16*>(smem + S * kPairStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * kPairStageBytes + kPairOutBytes);
+  uint64_t* empty = full + S;
+  uint64_t* accum = empty + S;
+  uint64_t* tmem_free = accum + 1;
+  uint64_t* drain = tmem_free + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t cta = ptx::cluster_ctarank();  // 0 issues the MMAs
+  const int cluster = blockIdx.x / 2, n_clusters = gridDim.x / 2;
+  const int n_tiles = (args.cols + kPairN - 1) / kPairN;  // token tiles
+  const int tiles = n_tiles * ((args.rows + 2 * kBM - 1) / (2 * kBM));
+  const bool has_d2 = args.kb2 > 0;
+  const int n1 = args.kb1;
+  const int per_tile = n1 + (has_d2 ? 2 * args.kb2 : 0);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], 1);
+    }
+    ptx::mbar_init(accum, 1);
+    ptx::mbar_init(tmem_free, 2 * kPairEpi / 32);  // one arrival per epilogue warp of both CTAs
+    ptx::mbar_init(drain, 1);
+    *abort_flag = prior_timeout(args.err);
+    ptx::fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(tmem_slot, kPairTmemCols);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  ptx::cluster_sync();  // both CTAs' barriers exist before either signals the other's
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  // programmatic dependent launch as in umma_kernel: after its own T = X.V
+  // kernel the forward streams W0 and X at once and waits before T
+  const bool early = args.early_start;
+  if (!early) asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  auto give_up = [&]() {
+    record_timeout(args.err);
+    *abort_flag = 1;
+  };
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------- producer (both CTAs)
+    ptx::prefetch_tmap(&tmA1);
+    ptx::prefetch_tmap(&tmB1);
+    const uint32_t full0 = ptx::mapa(ptx::smem_u32(full), 0);  // the MMA CTA's full barriers
+    bool waited = !early, stop = false;
+    int g = 0;  // stage items issued, over all tiles
+    for (int tile = cluster; tile < tiles && !stop; tile += n_clusters) {
+      const int row0 = (tile / n_tiles) * (2 * kBM) + (int)cta * kBM;
+      const int tok0 = (tile % n_tiles) * kPairN + (int)cta * kPairHalf;
+      for (int i = 0; i < per_tile; ++i, ++g) {
+        const int st = g % S;
+        const uint32_t ph = (uint32_t)(g / S) & 1u;
+        if (!ptx::mbar_wait(&empty[st], ph ^ 1u, abort_flag)) {
+          give_up();
+          stop = true;
+          break;
+        }
+        uint8_t* a = smem + st * kPairStageBytes;
+        uint8_t* b = a + kABytes;
+        if (cta == 0) ptx::mbar_arrive_expect_tx(&full[st], 2 * kPairStageBytes);  // both halves
+        const uint32_t bar = full0 + (uint32_t)(st * 8);
+        if (i < n1) {
+          ptx::tma_load_2d_pair(a, &tmA1, bar, i * kBK, row0);
+          ptx::tma_load_2d_pair(b, &tmB1, bar, i * kBK, tok0);
+        } else {
+          const int j = i - n1;
+          if (!waited) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            waited = true;
+          }
+          const int jx = (j % args.kb2) * kBK;
+          ptx::tma_load_2d_pair(a, &tmA2, bar, jx, row0);
+          ptx::tma_load_2d_pair(b, j < args.kb2 ? &tmB2 : &tmB3, bar, jx, tok0);
+        }
+      }
+    }
+    // drain: the MMAs that read a stage's last loads complete after those
+    // loads landed, and their commit reaches empty[] in both CTAs. After an
+    // abort, loads still in flight land within microseconds: wait a bounded
+    // tenth of a second for them without the abort shortcut.
+    for (int st = 0; st < S && st < g; ++st) {
+      const int last = st + ((g - 1 - st) / S) * S;
+      if (!ptx::mbar_wait(&empty[st], (uint32_t)(last / S) & 1u, abort_flag)) {
+        int never = 0;
+        ptx::mbar_wait(&empty[st], (uint32_t)(last / S) & 1u, &never, 100000000ull);
+      }
+    }
+  } else if (warp == 1 && lane == 0 && cta == 0) {
+    // ---------------------------------------------------------- MMA issuer (even CTA)
+    constexpr uint32_t idesc = ptx::idesc_bf16(2 * kBM, kPairN, 0);
+    bool stop = false;
+    int g = 0, j = 0, issued = 0;
+    for (int tile = cluster; tile < tiles; tile += n_clusters, ++j) {
+      // the epilogues of both CTAs have read the previous tile's accumulators
+      if (j > 0 && !ptx::mbar_wait(tmem_free, (uint32_t)(j - 1) & 1u, abort_flag)) {
+        give_up();
+        stop = true;
+        break;
+      }
+      ptx::tc_fence_after();
+      for (int i = 0; i < per_tile; ++i, ++g) {
+        const int st = g % S;
+        const uint32_t ph = (uint32_t)(g / S) & 1u;
+        if (!ptx::mbar_wait(&full[st], ph, abort_flag)) {
+          give_up();
+          stop = true;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t a = ptx::smem_u32(smem + st * kPairStageBytes);
+        const uint32_t b = a + kABytes;
+        // D1 = W0 . X^T over K = I at column 0; D2 = U . (T_hi + T_lo)^T at kPairN
+        const uint32_t d = i < n1 ? tmem : tmem + (uint32_t)kPairN;
+        const bool first = i == 0 || i == n1;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk)
+          ptx::umma_bf16_pair(d, ptx::sdesc_sw128(a + kk * 32, 16, 1024), ptx::sdesc_sw128(b + kk * 32, 16, 1024),
+                              idesc, (!first || kk > 0) ? 1u : 0u);
+        ptx::umma_commit_pair(&empty[st], kPairMask);
+        ++issued;
+      }
+      if (stop) break;
+      ptx::umma_commit_pair(accum, kPairMask);
+    }
+    if (stop && issued > 0) {
+      // aborted: the issued MMAs finish before tensor memory is released
+      ptx::umma_commit_pair(drain, 0x1);
+      int never = 0;
+      ptx::mbar_wait(drain, 0, &never);
+    }
+  } else if (warp >= 2) {
+    // ---------------------------------------------------------- epilogue (both CTAs)
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;  // accumulator row = TMEM lane
+    const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
+    const bool storer = threadIdx.x == 64;  // issues the TMA stores of the tile
+    const uint32_t free_bar = ptx::mapa(ptx::smem_u32(tmem_free), 0);
+    if (early) asm volatile("griddepcontrol.wait;" ::: "memory");
+    bool ok = true;
+    int j = 0;
+    for (int tile = cluster; tile < tiles; tile += n_clusters, ++j) {
+      const int row0 = (tile / n_tiles) * (2 * kBM) + (int)cta * kBM;
+      const int col0 = (tile % n_tiles) * kPairN;
+      const int ncols = min(kPairN, args.cols - col0);
+      if (storer) ptx::bulk_wait_read();  // the previous tile's store has read sOut
+      const bool got = ptx::mbar_wait(accum, (uint32_t)j & 1u, abort_flag);
+      // one decision for all four warps: the barriers below need every one of them
+      ok = ptx::bar_red_and(1, kPairEpi, got);
+      if (!ok) break;
+      ptx::tc_fence_after();
+      const int grow = row0 + row;
+      const float so = (grow < args.rows) ? __ldg(args.s + grow) : 0.f;
+      for (int c0 = 0; c0 < ncols; c0 += 16) {
+        float d1[16], d2[16];
+        ptx::tmem_ld16(taddr + c0, d1);
+        if (has_d2) ptx::tmem_ld16(taddr + kPairN + c0, d2);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          sOut[(c0 + e) * kBM + row] = __float2bfloat16_rn(has_d2 ? fmaf(so, d1[e], d2[e]) : so * d1[e]);
+      }
+      // tensor memory read: the next tile's MMAs may start
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive_cluster(free_bar);
+      ptx::fence_proxy_async_smem();
+      asm volatile("bar.sync 1, %0;" ::"n"(kPairEpi) : "memory");
+      if (storer) {
+        // rows past O and tokens past M fall outside Y and are not written
+        ptx::tma_store_2d(&tmY, sOut, row0, col0);
+        ptx::bulk_commit();
+      }
+    }
+    if (!ok && !*abort_flag) give_up();
+    if (storer) ptx::bulk_wait_all();
+  }
+
+  __syncwarp();
+  ptx::tc_fence_before();
+  ptx::cluster_sync();  // both epilogues have read their accumulators; every MMA has completed
+  if (warp == 1) ptx::tmem_dealloc_pair(tmem, kPairTmemCols);
+}
+
 // s (.) W0 for rank 0 (no tensor-core work).
 __global__ void __launch_bounds__(256) scale_rows_kernel(const float* __restrict__ s, const bf16* __restrict__ W0,
                                                          int64_t I, int64_t nvec, bf16* __restrict__ out) {
@@ -694,15 +925,18 @@ recon_band_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constan
     const int row = quarter * 32 + lane;  // tensor-memory lane = row of the tile
     const uint32_t taddr0 = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(half * 64);
     const bool leader = threadIdx.x == 64;  // issues the stores
-    bool ok = ptx::mbar_wait(w_full, 0, abort_flag);
+    // Every decision to stop is taken by all eight epilogue warps together
+    // (bar.red.and): the named barriers below need every one of them, and
+    // tcgen05.ld is warp-collective. A wait can succeed in one warp and give
+    // up in another when an abort lands just as the barrier completes.
+    bool ok = ptx::bar_red_and(1, kBandEpi, ptx::mbar_wait(w_full, 0, abort_flag));
     for (int l = 0; l < n && ok; ++l) {
       const int b = l & 1;
       const uint32_t taddr = taddr0 + (uint32_t)(b * kRecN);
-      ok = ptx::mbar_wait(&acc_full[b], (uint32_t)((l >> 1) & 1), abort_flag);
+      const bool got = ptx::mbar_wait(&acc_full[b], (uint32_t)((l >> 1) & 1), abort_flag);
       // the store of layer l - kOutBufs read its buffer before this layer rewrites it
       if (leader) ptx::bulk_wait_read_n<C::kOutBufs - 1>();
-      ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld is warp-collective
-      asm volatile("bar.sync 1, %0;" ::"n"(kBandEpi) : "memory");
+      ok = ptx::bar_red_and(1, kBandEpi, got);
       if (!ok) break;
       ptx::tc_fence_after();
       const float so = (o0 + row < a.O) ? __ldg(a.s[l] + o0 + row) : 0.f;
@@ -763,23 +997,29 @@ EncodeTiledFn encode_fn(cudaError_t* e) {
   return fn;
 }
 
-// 2-D bf16 tensor [rows, cols], row pitch = cols, box [box_rows, 64] with
-// 128-byte swizzle; out-of-bounds elements of a box read as zero.
-int make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows, cudaError_t* ce) {
+// 2-D bf16 tensor [rows, cols], row pitch = cols, box [box_rows, box_cols];
+// out-of-bounds elements of a box read as zero and are not written.
+int make_map_box(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows, int box_cols,
+                 CUtensorMapSwizzle swizzle, cudaError_t* ce) {
   EncodeTiledFn enc = encode_fn(ce);
   if (!enc) return THETA_ERR_CUDA;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)box_rows};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     *ce = cudaErrorInvalidValue;
     return THETA_ERR_CUDA;
   }
   return THETA_OK;
+}
+
+// The operand layout of the MMA kernels: box [box_rows, 64], 128-byte swizzle.
+int make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows, cudaError_t* ce) {
+  return make_map_box(m, base, rows, cols, box_rows, kBK, CU_TENSOR_MAP_SWIZZLE_128B, ce);
 }
 
 // Per-device, per-kernel launch configuration: dynamic shared memory opt-in,
@@ -893,6 +1133,43 @@ cudaError_t launch_tile_kernel(const LaunchCtx& c, const Maps& mp, Args args, in
                     : pick_splits(tiles, args.kb1, capacity, info[c.device].max_cluster);
   return launch_pdl(kern, dim3((unsigned)(n_tiles * args.splits), (unsigned)m_tiles, 1), dim3(kThreads), C::kSmemBytes,
                     c.stream, args.splits, mp.a1, mp.b1, mp.a2, mp.b2, mp.b3, mp.a1u, mp.a2u, mp.b2u, mp.b3u, args);
+}
+
+// The persistent CTA-pair forward: one cluster of two per pair of SMs that
+// can hold one (the occupancy query, once per device), at most one per tile.
+cudaError_t launch_pair_forward(const LaunchCtx& c, const Maps& mp, const CUtensorMap& mY, const Args& args,
+                                int64_t tiles) {
+  auto kern = pair_forward_kernel;
+  static KernelInfo info[64];
+  static int max_clusters[64];
+  cudaError_t e = prepare_kernel(&info[c.device], c.device, kern, kThreads, kPairSmemBytes, kPairTmemCols, false);
+  if (e != cudaSuccess) return e;
+  {
+    std::lock_guard<std::mutex> lk(setup_mutex());
+    if (max_clusters[c.device] == 0) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(2, 1, 1);
+      cfg.blockDim = dim3(kThreads, 1, 1);
+      cfg.dynamicSmemBytes = kPairSmemBytes;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = 2;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      const bool pending = cudaPeekAtLastError() != cudaSuccess;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) {
+        if (!pending) cudaGetLastError();  // a refused query is not an error of this call
+        n = c.num_sms / 2;                 // one CTA per SM
+      }
+      max_clusters[c.device] = n;
+    }
+  }
+  const int64_t clusters = tiles < max_clusters[c.device] ? tiles : max_clusters[c.device];
+  return launch_pdl(kern, dim3((unsigned)(2 * clusters), 1, 1), dim3(kThreads), kPairSmemBytes, c.stream, 2, mp.a1,
+                    mp.b1, mp.a2, mp.b2, mp.b3, mY, args);
 }
 
 template <int KB>
@@ -1011,13 +1288,18 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
   const int BN = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 256 ? 128 : 256;
   const int m_tiles = (int)ceil_div(O, kBM);
   const int n_tiles = (int)ceil_div(M, BN);
+  // More than 256 tokens: pairs of SMs share 256 x 256 tiles whenever every
+  // CTA gets a whole tile -- under the throughput policy, or when the tiles
+  // already fill the GPU (the latency policy would not split K then either).
+  const bool pair = BN == 256 && (c.policy == THETA_POLICY_THROUGHPUT || (int64_t)m_tiles * n_tiles >= c.num_sms);
+  const int box_b = pair ? kPairHalf : BN;  // tokens per B box
   Maps mp;
   if ((st = make_map(&mp.a1, W0, O, I, kBM, ce))) return st;
-  if ((st = make_map(&mp.b1, X, M, I, BN, ce))) return st;
+  if ((st = make_map(&mp.b1, X, M, I, box_b, ce))) return st;
   if (r > 0) {
     if ((st = make_map(&mp.a2, U, O, r, kBM, ce))) return st;
-    if ((st = make_map(&mp.b2, t_hi, M, r, BN, ce))) return st;
-    if ((st = make_map(&mp.b3, t_lo, M, r, BN, ce))) return st;
+    if ((st = make_map(&mp.b2, t_hi, M, r, box_b, ce))) return st;
+    if ((st = make_map(&mp.b3, t_lo, M, r, box_b, ce))) return st;
   } else {
     mp.a2 = mp.a1;
     mp.b2 = mp.b3 = mp.b1;
@@ -1033,6 +1315,18 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
   a.out = static_cast<bf16*>(Y);
   a.early_start = r > 0;  // directly after this call's T = X.V kernel
   a.err = c.err;
+  if (pair) {
+    a.splits = 1;
+    // Y [M, O] written by TMA: boxes of 128 rows of W0 (columns of Y) x 256 tokens
+    CUtensorMap mY;
+    if ((st = make_map_box(&mY, Y, M, O, kPairN, kBM, CU_TENSOR_MAP_SWIZZLE_NONE, ce))) return st;
+    e = launch_pair_forward(c, mp, mY, a, ceil_div(O, 2 * kBM) * ceil_div(M, kPairN));
+    if (e != cudaSuccess) {
+      *ce = e;
+      return THETA_ERR_CUDA;
+    }
+    return THETA_OK;
+  }
   switch (BN) {
     case 16: e = launch_tile_kernel<16, MODE_FORWARD>(c, mp, a, m_tiles, n_tiles); break;
     case 32: e = launch_tile_kernel<32, MODE_FORWARD>(c, mp, a, m_tiles, n_tiles); break;

@@ -114,6 +114,43 @@ def test_forward_throughput_policy(lib, torch, M, O, I, r):
     assert_close(got, ref, "bf16", "Y")
 
 
+# More than 256 tokens with a whole tile per CTA: pairs of SMs share 256 x 256
+# tiles (the even CTA's MMAs read both CTAs' halves of W0 and X). Ragged row
+# pairs (the odd CTA's rows partly or wholly past O), ragged token tiles (the
+# odd CTA's tokens wholly past M), K not a multiple of 64, rank 0 and the
+# largest rank.
+PAIR_CASES = [
+    (600, 392, 328, 64),     # 1.5 row pairs, 2.3 token tiles
+    (257, 264, 1160, 40),    # one token in the second tile
+    (520, 1032, 264, 0),     # rank 0: no D2
+    (300, 264, 392, 256),    # four rank blocks, hi and lo parts each
+    (2100, 520, 1096, 16),
+]
+
+
+@pytest.mark.parametrize("M,O,I,r", PAIR_CASES)
+def test_forward_pair_tiles(lib, torch, M, O, I, r):
+    X, W0, s, U, V = bundle(M, O, I, r, "bf16", seed=M + O)
+    ref = oracle.linear_forward(X, W0, s, U, V)
+    lib.theta_set_policy(lib.THETA_POLICY_THROUGHPUT)
+    try:
+        got = run_forward(lib, torch, X, W0, s, U, V, "bf16")
+    finally:
+        lib.theta_set_policy(lib.THETA_POLICY_LATENCY)
+    assert_close(got, ref, "bf16", f"Y {M}x{O}x{I} r{r}")
+
+
+def test_forward_pair_tiles_fill_the_gpu_under_latency_policy(lib, torch):
+    """Under the latency policy the pair path is taken once the 128 x 256
+    tiles alone fill the GPU (here 26 x 6 = 156 tiles)."""
+    M, O, I, r = 1300, 3208, 1160, 40
+    X, W0, s, U, V = bundle(M, O, I, r, "bf16", seed=13)
+    got = run_forward(lib, torch, X, W0, s, U, V, "bf16")
+    rows = np.r_[0:8, 120:136, 250:262, 1500:1530, 3190:3208]
+    ref = oracle.linear_forward(X, W0[rows], s[rows], U[rows], V)
+    assert_close(got[:, rows], ref, "bf16", "Y")
+
+
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
 def test_forward_rank0_is_scaled_shared_block(lib, torch, dt):
     X, W0, s, U, V = bundle(9, 264, 520, 0, dt, seed=3)

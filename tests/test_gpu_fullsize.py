@@ -83,7 +83,7 @@ def test_gemma3_1b_family_all_stages(lib, torch, fam):
 
 
 @pytest.mark.parametrize("fam,M", [("gate", 1), ("gate", 4), ("gate", 64), ("gate", 2048), ("k", 1), ("k", 2), ("q", 2),
-                                   ("down", 1), ("down", 3), ("down", 16), ("o", 256)])
+                                   ("down", 1), ("down", 3), ("down", 16), ("down", 2048), ("o", 256)])
 def test_gemma4_31b_forward(lib, torch, fam, M):
     O, I = syn.GEMMA4_31B.shapes[fam]
     r = 64
