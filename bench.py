@@ -278,7 +278,7 @@ KERNEL_NAMES = {
     "frob": "frob_partial_kernel + frob_final_kernel",
     "forward_decode": "gemv_rows_kernel / grouped_rows_kernel / umma_kernel<16..64,FORWARD>",
     "forward_ridge": "umma_kernel<128,FORWARD> (+ umma_kernel<64,XV>)",
-    "forward_prefill": "umma_kernel<256,FORWARD> (+ umma_kernel<64,XV>)",
+    "forward_prefill": "pair_kernel<FORWARD> (+ umma_kernel<64,XV>)",
 }
 
 
@@ -963,6 +963,9 @@ def run_op(args):
     torch.cuda.set_device(0)
     import linear_theta_forward_b200 as theta
     peaks = measured_peaks()
+    # the step runs under the throughput policy; single ops default to latency
+    theta.theta_set_policy(theta.THETA_POLICY_THROUGHPUT if args.policy == "throughput"
+                           else theta.THETA_POLICY_LATENCY)
     M, O, I, r, L, G = args.M, args.O, args.I, args.rank, args.layers, args.G
     seed = 0
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
@@ -1164,7 +1167,7 @@ def run_op(args):
         l2 = "flushed (256 MiB write) before every call (median of %d)" % len(per_call)
     theta.theta_device_status()
     line = {"op": args.op, "shape": {"M": M, "O": O, "I": I, "rank": r, "layers": L, "G": G}, "dtype": "bf16",
-            "ms": round(ms, 5), "iters": args.iters, "l2": l2,
+            "ms": round(ms, 5), "iters": args.iters, "l2": l2, "policy": args.policy,
             "GB/s": round(nbytes / (ms * 1e-3) / 1e9, 1),
             "frac_hbm": round(nbytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4), "algorithmic_bytes": nbytes,
             "clocks": clocks.summary()}
@@ -1198,6 +1201,8 @@ def main(argv=None):
                                      "prelude", "frob", "svd"],
                     help="time one entry point on one problem instead of the whole step")
     ap.add_argument("--model", choices=["1b", "31b"], default="31b", help="--op layer_forward: the model's shapes")
+    ap.add_argument("--policy", choices=["latency", "throughput"], default="latency",
+                    help="--op: the library's launch policy (the step uses throughput)")
     ap.add_argument("--M", type=int, default=256)
     ap.add_argument("--O", type=int, default=21504)
     ap.add_argument("--I", type=int, default=5376)

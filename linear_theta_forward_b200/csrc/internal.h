@@ -91,6 +91,17 @@ bool launch_forward_nvfp4(const LaunchCtx& c, const void* X, const void* codes, 
 // ---- randomized SVD of a residual (svd_kernels.cu): R [O, I] in dt, omega
 // fp32 [samples, I]; U [O, rank], V [I, rank] in dt; ws of svd_workspace_bytes.
 int svd_max_samples();
+// Tensor-core products of a bf16 residual R [O, I] with an fp32 factor given
+// as three bf16 parts, part_stride elements apart (umma_kernels.cu). r_left:
+// part_out[z] = R . F^T [O, k], F parts [k, I] (row pitch I); otherwise
+// part_out[z] = F^T . R [k, I], parts of Q^T [k, O] with row pitch
+// part_pitch (a multiple of 8). Split z of `splits`
+// (at most kSvdMaxSplits, from svd_mma_splits) covers a fixed share of K;
+// the caller sums the splits. Needs I % 8 == 0 and 16-byte aligned R.
+constexpr int kSvdMaxSplits = 8;
+int svd_mma_splits(const LaunchCtx& c, bool r_left, int64_t O, int64_t I, int k);
+int launch_svd_mma(const LaunchCtx& c, bool r_left, const void* R, int64_t O, int64_t I, const void* parts,
+                   int64_t part_stride, int64_t part_pitch, int k, int splits, float* part_out, cudaError_t* ce);
 size_t svd_workspace_bytes(int64_t O, int64_t I, int samples, int rank);
 cudaError_t launch_residual_svd(const LaunchCtx& c, theta_dtype dt, const void* R, int64_t O, int64_t I, int rank,
                                 int samples, int power_iters, const float* omega, void* U, void* V, void* ws);

@@ -30,6 +30,7 @@ constexpr int kT = 256;           // threads of the tile GEMM
 constexpr int kBM = 64, kBK = 16;  // output tile edge, K per shared-memory step
 constexpr int kChain = 256;        // products per fp32 partial sum
 constexpr int kMaxSamples = 96;    // k: the one-CTA fp64 steps hold two k x k matrices
+constexpr int kSvdParts3 = 3;      // bf16 parts of an fp32 factor on the tensor-core products
 
 template <typename T>
 __device__ __forceinline__ float ldf(const T* p, int64_t i) {
@@ -106,6 +107,43 @@ gemm_kernel(const TA* __restrict__ A, const TB* __restrict__ B, int64_t M, int64
       const int64_t n = n0 + tx + 16 * j;
       if (n < N) Cz[m * N + n] = acc[i][j] + part[i][j];
     }
+  }
+}
+
+// The exact split of an fp32 value into three bf16 parts, x = p1 + p2 + p3:
+// each part is the remainder so far rounded to bf16, and each remainder is
+// exact in fp32 (x - p1 and its successor lose no bits).
+__device__ __forceinline__ void split3(float x, bf16* p) {
+  const bf16 a = __float2bfloat16_rn(x);
+  const float r1 = x - __bfloat162float(a);
+  const bf16 b = __float2bfloat16_rn(r1);
+  const float r2 = r1 - __bfloat162float(b);
+  p[0] = a, p[1] = b, p[2] = __float2bfloat16_rn(r2);
+}
+
+// F [rows, cols] fp32 -> parts [3][rows, cols] bf16 (each part_elems apart)
+__global__ void __launch_bounds__(256) split3_kernel(const float* __restrict__ F, int64_t count,
+                                                     bf16* __restrict__ parts, int64_t part_elems) {
+  pdl_enter(F, parts);
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
+    bf16 p[3];
+    split3(F[i], p);
+    parts[i] = p[0], parts[part_elems + i] = p[1], parts[2 * part_elems + i] = p[2];
+  }
+}
+
+// Q [O, k] fp32 -> parts of Q^T: [3][k, pitch] bf16, element (j, o) = Q[o, j]
+__global__ void __launch_bounds__(256) split3_transpose_kernel(const float* __restrict__ Q, int64_t O, int k,
+                                                               bf16* __restrict__ parts, int64_t pitch,
+                                                               int64_t part_elems) {
+  pdl_enter(Q, parts);
+  const int64_t count = O * k;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t j = i / O, o = i % O;  // consecutive threads write consecutive o
+    bf16 p[3];
+    split3(Q[o * k + j], p);
+    const int64_t d = j * pitch + o;
+    parts[d] = p[0], parts[part_elems + d] = p[1], parts[2 * part_elems + d] = p[2];
   }
 }
 
@@ -362,8 +400,10 @@ size_t small_smem(int k) { return (size_t)2 * k * k * sizeof(double); }
 struct SvdPlan {
   int64_t O, I;
   int k, r;
+  int64_t qpitch;  // row pitch (elements) of the parts of Q^T [k, O]
+  int64_t part_elems;  // elements per bf16 part of F
   // workspace offsets, in floats
-  int64_t y0, y1, z0, z1, bm, g, li, lit, s, e, et, uraw, vun, sig, part, total;
+  int64_t y0, y1, z0, z1, bm, g, li, lit, s, e, et, uraw, vun, sig, part, parts, total;
 };
 
 SvdPlan plan_svd(int64_t O, int64_t I, int k, int r) {
@@ -393,9 +433,45 @@ SvdPlan plan_svd(int64_t O, int64_t I, int k, int r) {
   need(k, I, k);  // L^-1 Z^T
   need(O, r, k);  // Q E_r
   need(I, r, k);  // B^T E_r
+  // the tensor-core products with a bf16 R: split partials of C [O, k] or
+  // [k, I], and the three bf16 parts of the fp32 factor
+  const int64_t mma_part = (int64_t)kSvdMaxSplits * (O * k > k * I ? O * k : k * I);
+  if (mma_part > part) part = mma_part;
   p.part = take(part > 0 ? part : 1);
+  p.qpitch = (O + 7) / 8 * 8;
+  p.part_elems = (int64_t)k * (p.qpitch > I ? p.qpitch : I);
+  p.parts = take((kSvdParts3 * p.part_elems + 1) / 2);
   p.total = at;
   return p;
+}
+
+// One product of the bf16 residual with an fp32 factor on tensor cores (the
+// factor split into three bf16 parts, the K splits summed in order).
+// r_left: out [O, k] = R . F^T, F [k, I]; else out [k, I] = Q^T . R, Q [O, k].
+cudaError_t product_mma(const LaunchCtx& c, const SvdPlan& p, float* ws, bool r_left, const bf16* R,
+                        const float* F, float* out) {
+  const int64_t O = p.O, I = p.I;
+  const int k = p.k;
+  bf16* parts = reinterpret_cast<bf16*>(ws + p.parts);
+  const auto blocks = [&](int64_t n) {
+    int64_t b = ceil_div(n, 256);
+    return (unsigned)(b > 8 * (int64_t)c.num_sms ? 8 * (int64_t)c.num_sms : b);
+  };
+  cudaError_t e = r_left ? launch_pdl(split3_kernel, dim3(blocks(k * I)), dim3(256), 0, c.stream, 1, F, (int64_t)k * I,
+                                      parts, p.part_elems)
+                         : launch_pdl(split3_transpose_kernel, dim3(blocks(O * k)), dim3(256), 0, c.stream, 1, F, O,
+                                      k, parts, p.qpitch, p.part_elems);
+  if (e != cudaSuccess) return e;
+  const int sp = svd_mma_splits(c, r_left, O, I, k);
+  float* dst = sp > 1 ? ws + p.part : out;
+  int st = launch_svd_mma(c, r_left, R, O, I, parts, p.part_elems, r_left ? I : p.qpitch, k, sp, dst, &e);
+  if (st != THETA_OK) return e != cudaSuccess ? e : cudaErrorInvalidValue;
+  if (sp == 1) return cudaSuccess;
+  const int64_t count = r_left ? O * k : (int64_t)k * I;
+  int64_t nb = ceil_div(count, 256);
+  if (nb > 4 * (int64_t)c.num_sms) nb = 4 * (int64_t)c.num_sms;
+  return launch_pdl(sum_splits_kernel, dim3((unsigned)nb), dim3(256), 0, c.stream, 1, (const float*)(ws + p.part), sp,
+                    count, out);
 }
 
 // C = op(A) . op(B)^T with the split and its fixed-order sum; out fp32 [M, N]
@@ -478,20 +554,34 @@ cudaError_t run_svd(const LaunchCtx& c, const T* R, int64_t O, int64_t I, int r,
   float* part = ws + p.part;
   float *Y = ws + p.y0, *Ytmp = ws + p.y1, *Zt = ws + p.z0, *Ztmp = ws + p.z1, *Bm = ws + p.bm;
   float* Q;
+  // The products that stream R: on tensor cores for a bf16 R whose rows TMA
+  // can address (16-byte aligned, I a multiple of 8), else CUDA-core tiles.
+  bool mma = false;
+  if constexpr (sizeof(T) == 2) mma = I % 8 == 0 && (reinterpret_cast<uintptr_t>(R) & 15u) == 0;
+  auto r_times = [&](const float* F, float* out) -> cudaError_t {  // out [O, k] = R . F^T
+    if constexpr (sizeof(T) == 2)
+      if (mma) return product_mma(c, p, ws, true, R, F, out);
+    return gemm<T, float, false, false>(c, R, F, O, k, I, out, part);
+  };
+  auto qt_times_r = [&](const float* Qm, float* out) -> cudaError_t {  // out [k, I] = Q^T . R
+    if constexpr (sizeof(T) == 2)
+      if (mma) return product_mma(c, p, ws, false, R, Qm, out);
+    return gemm<float, T, true, true>(c, Qm, R, k, I, O, out, part);
+  };
   // range sample and its orthonormal basis
-  if ((e = gemm<T, float, false, false>(c, R, omega, O, k, I, Y, part))) return e;  // Y = R Omega^T
+  if ((e = r_times(omega, Y))) return e;  // Y = R Omega^T
   if ((e = orth_cols(c, p, ws, O, Y, Ytmp, &Q))) return e;
   for (int it = 0; it < power_iters; ++it) {
     float* Qz;
-    if ((e = gemm<float, T, true, true>(c, Q, R, k, I, O, Zt, part))) return e;  // Zt = Q^T R
+    if ((e = qt_times_r(Q, Zt))) return e;  // Zt = Q^T R
     if ((e = orth_rows(c, p, ws, I, Zt, Ztmp, &Qz))) return e;
     float* Ynext = (Q == Y) ? Ytmp : Y;
-    if ((e = gemm<T, float, false, false>(c, R, Qz, O, k, I, Ynext, part))) return e;  // Y = R Z
+    if ((e = r_times(Qz, Ynext))) return e;  // Y = R Z
     float* other = (Ynext == Y) ? Ytmp : Y;
     if ((e = orth_cols(c, p, ws, O, Ynext, other, &Q))) return e;
   }
   // projection, its small SVD through B B^T, and the lift
-  if ((e = gemm<float, T, true, true>(c, Q, R, k, I, O, Bm, part))) return e;              // B = Q^T R
+  if ((e = qt_times_r(Q, Bm))) return e;  // B = Q^T R
   if ((e = gemm<float, float, false, false>(c, Bm, Bm, k, k, I, ws + p.s, part))) return e;  // B B^T
   if ((e = launch_pdl(jacobi_eig_kernel, dim3(1), dim3(256), small_smem(k), c.stream, 1, (const float*)(ws + p.s), k,
                       r, ws + p.e, ws + p.et)))

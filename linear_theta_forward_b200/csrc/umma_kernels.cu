@@ -380,47 +380,66 @@ umma_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CU
   if (warp == 1) ptx::tmem_dealloc(tmem, C::kTmemCols);
 }
 
-// ------------------------------------------------------------ CTA-pair forward
-// The FORWARD epilogue over 256 x 256 tiles (weight rows x tokens) on pairs
-// of SMs: the two CTAs of a cluster of two share each tcgen05 MMA of M = 256,
-// N = 256 (cta_group::2), issued by the even CTA. Each CTA stages its own half
-// of both operands -- 128 weight rows and 128 tokens, 32 KB per 64-wide K
-// block -- and receives its 128 rows x 256 tokens of D1 and D2 in its own
-// tensor memory. Per K block an SM takes in two thirds of what a 128 x 256
-// tile on one SM does for the same tensor work.
+// ------------------------------------------------------------ CTA-pair tiles
+// The FORWARD and GATE_UP epilogues over 256-row tiles on pairs of SMs: the
+// two CTAs of a cluster of two share each tcgen05 MMA of M = 256 weight rows
+// (cta_group::2), issued by the even CTA. Each CTA stages its own half of
+// both operands -- 128 weight rows (of each projection) and half the tile's
+// tokens per 64-wide K block -- and receives its 128 rows of every
+// accumulator in its own tensor memory. FORWARD tiles are 256 tokens wide
+// (D1, D2: 2 x 256 columns), GATE_UP tiles 128 (D1 and D2 of the gate and of
+// the up projection: 4 x 128 columns). Per K block an SM takes in two thirds
+// (FORWARD) or five sixths (GATE_UP) of what a one-SM tile of the same
+// tensor work does.
 //
 // The kernel is persistent: a cluster walks the tiles c, c + clusters, ...
 // Its producers load the next tile's stages while the epilogue still works
 // on the current one, and the epilogue hands tensor memory back as soon as it
-// has moved the tile into shared memory (s * D1 + D2, rounded to bf16, as
-// [token][row] -- the layout of Y), before one TMA store writes it out. So
-// between two tiles the tensor pipe waits only for that drain, not for a CTA
-// to finish, launch and fill its pipeline.
+// has moved the tile into shared memory (rounded to bf16 as [token][row], the
+// layout of Y), before one TMA store writes it out. So between two tiles the
+// tensor pipe waits only for that drain, not for a CTA to finish, launch and
+// fill its pipeline.
 //
 // Each CTA's producer signals the even CTA's full barrier (which expects
 // both halves); MMA completion is committed to the empty and accumulator
 // barriers of both CTAs; the epilogue warps of both CTAs arrive on the even
 // CTA's tensor-memory-free barrier.
-constexpr int kPairN = 256;                                     // tokens per pair tile: MMA N
-constexpr int kPairHalf = kPairN / 2;                           // tokens staged by each CTA
-constexpr int kPairStageBytes = kABytes + kPairHalf * kBK * 2;  // 16 KB of W0 (or U) + 16 KB of X (or T)
-constexpr int kPairStages = 5;
-constexpr int kPairOutBytes = kBM * kPairN * 2;                 // a CTA's Y tile, bf16 [token][row]
-constexpr int kPairTmemCols = 2 * kPairN;                       // D1, D2
-constexpr int kPairSmemBytes = kPairStages * kPairStageBytes + kPairOutBytes + 1024 /*align*/ + 256 /*barriers*/;
-constexpr uint16_t kPairMask = 0x3;                             // both CTAs of the cluster
-constexpr int kPairEpi = 128;                                   // epilogue threads per CTA
+template <int MODE>
+struct PairCfg {
+  static constexpr int kNumA = MODE == MODE_GATE_UP ? 2 : 1;  // weight tiles per phase-1 stage
+  static constexpr int kN = MODE == MODE_GATE_UP ? 128 : 256;  // tokens per tile: MMA N
+  static constexpr int kHalf = kN / 2;                         // tokens staged by each CTA
+  static constexpr int kBBytes = kHalf * kBK * 2;
+  static constexpr int kStageBytes = kNumA * kABytes + kBBytes;
+  static constexpr int kStages = MODE == MODE_GATE_UP ? 4 : 5;
+  static constexpr int kOutBytes = kBM * kN * 2;  // a CTA's Y tile, bf16 [token][row]
+  static constexpr int kTmemCols = 2 * kNumA * kN;  // D1 (per projection), then D2 (per projection)
+  static_assert(kTmemCols == 512, "the accumulators fill tensor memory");
+  static constexpr int kSmemBytes = kStages * kStageBytes + kOutBytes + 1024 /*align*/ + 256 /*barriers*/;
+  // warps 0 (TMA) and 1 (MMA), then the epilogue: one warp per 32-lane
+  // quarter of tensor memory for FORWARD; two for GATE_UP, each draining half
+  // of the tile's columns, since its GELU makes the drain several times
+  // longer (measured: eight warps slow the forward by 5%, speed gate/up up)
+  static constexpr int kEpiWarps = MODE == MODE_GATE_UP ? 8 : 4;
+  static constexpr int kEpi = 32 * kEpiWarps;
+  static constexpr int kThreads = 64 + kEpi;
+};
+constexpr uint16_t kPairMask = 0x3;  // both CTAs of the cluster
 
-__global__ void __launch_bounds__(kThreads)
-pair_forward_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
-                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
-                    const __grid_constant__ CUtensorMap tmB3, const __grid_constant__ CUtensorMap tmY,
-                    const Args args) {
-  constexpr int S = kPairStages;
+template <int MODE>
+__global__ void __launch_bounds__(PairCfg<MODE>::kThreads)
+pair_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+            const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+            const __grid_constant__ CUtensorMap tmB3, const __grid_constant__ CUtensorMap tmA1u,
+            const __grid_constant__ CUtensorMap tmA2u, const __grid_constant__ CUtensorMap tmB2u,
+            const __grid_constant__ CUtensorMap tmB3u, const __grid_constant__ CUtensorMap tmY, const Args args) {
+  using C = PairCfg<MODE>;
+  constexpr int S = C::kStages;
+  constexpr int N = C::kN;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  bf16* sOut = reinterpret_cast<bf16*>(smem + S * kPairStageBytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * kPairStageBytes + kPairOutBytes);
+  bf16* sOut = reinterpret_cast<bf16*>(smem + S * C::kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kOutBytes);
   uint64_t* empty = full + S;
   uint64_t* accum = empty + S;
   uint64_t* tmem_free = accum + 1;
@@ -431,11 +450,11 @@ pair_forward_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_const
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const uint32_t cta = ptx::cluster_ctarank();  // 0 issues the MMAs
   const int cluster = blockIdx.x / 2, n_clusters = gridDim.x / 2;
-  const int n_tiles = (args.cols + kPairN - 1) / kPairN;  // token tiles
+  const int n_tiles = (args.cols + N - 1) / N;  // token tiles
   const int tiles = n_tiles * ((args.rows + 2 * kBM - 1) / (2 * kBM));
   const bool has_d2 = args.kb2 > 0;
   const int n1 = args.kb1;
-  const int per_tile = n1 + (has_d2 ? 2 * args.kb2 : 0);
+  const int per_tile = n1 + (has_d2 ? 2 * C::kNumA * args.kb2 : 0);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -443,13 +462,13 @@ pair_forward_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_const
       ptx::mbar_init(&empty[i], 1);
     }
     ptx::mbar_init(accum, 1);
-    ptx::mbar_init(tmem_free, 2 * kPairEpi / 32);  // one arrival per epilogue warp of both CTAs
+    ptx::mbar_init(tmem_free, 2 * C::kEpiWarps);  // one arrival per epilogue warp of both CTAs
     ptx::mbar_init(drain, 1);
     *abort_flag = prior_timeout(args.err);
     ptx::fence_mbarrier_init();
   }
   if (warp == 1) {
-    ptx::tmem_alloc_pair(tmem_slot, kPairTmemCols);
+    ptx::tmem_alloc_pair(tmem_slot, C::kTmemCols);
     ptx::tmem_relinquish_pair();
   }
   ptx::tc_fence_before();
@@ -457,7 +476,7 @@ pair_forward_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_const
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // programmatic dependent launch as in umma_kernel: after its own T = X.V
-  // kernel the forward streams W0 and X at once and waits before T
+  // kernels the forward streams W0 and X at once and waits before T
   const bool early = args.early_start;
   if (!early) asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -476,7 +495,7 @@ pair_forward_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_const
     int g = 0;  // stage items issued, over all tiles
     for (int tile = cluster; tile < tiles && !stop; tile += n_clusters) {
       const int row0 = (tile / n_tiles) * (2 * kBM) + (int)cta * kBM;
-      const int tok0 = (tile % n_tiles) * kPairN + (int)cta * kPairHalf;
+      const int tok0 = (tile % n_tiles) * N + (int)cta * C::kHalf;
       for (int i = 0; i < per_tile; ++i, ++g) {
         const int st = g % S;
         const uint32_t ph = (uint32_t)(g / S) & 1u;
@@ -485,22 +504,45 @@ pair_forward_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_const
           stop = true;
           break;
         }
-        uint8_t* a = smem + st * kPairStageBytes;
-        uint8_t* b = a + kABytes;
-        if (cta == 0) ptx::mbar_arrive_expect_tx(&full[st], 2 * kPairStageBytes);  // both halves
+        uint8_t* a = smem + st * C::kStageBytes;
+        uint8_t* b = a + C::kNumA * kABytes;
         const uint32_t bar = full0 + (uint32_t)(st * 8);
-        if (i < n1) {
+        if constexpr (MODE == MODE_FORWARD) {
+          // both halves; phase-1 and phase-2 items move the same bytes
+          if (cta == 0) ptx::mbar_arrive_expect_tx(&full[st], 2 * C::kStageBytes);
+          if (i < n1) {
+            ptx::tma_load_2d_pair(a, &tmA1, bar, i * kBK, row0);
+            ptx::tma_load_2d_pair(b, &tmB1, bar, i * kBK, tok0);
+          } else {
+            const int j = i - n1;
+            if (!waited) {
+              asm volatile("griddepcontrol.wait;" ::: "memory");
+              waited = true;
+            }
+            const int jx = (j % args.kb2) * kBK;
+            ptx::tma_load_2d_pair(a, &tmA2, bar, jx, row0);
+            ptx::tma_load_2d_pair(b, j < args.kb2 ? &tmB2 : &tmB3, bar, jx, tok0);
+          }
+        } else if (i < n1) {
+          // both halves: every weight tile and the token tile of each CTA
+          if (cta == 0) ptx::mbar_arrive_expect_tx(&full[st], 2 * C::kStageBytes);
           ptx::tma_load_2d_pair(a, &tmA1, bar, i * kBK, row0);
+          ptx::tma_load_2d_pair(a + kABytes, &tmA1u, bar, i * kBK, row0);
           ptx::tma_load_2d_pair(b, &tmB1, bar, i * kBK, tok0);
         } else {
+          // one U tile and one part of T: (high, low) of the gate projection,
+          // then (high, low) of the up projection
           const int j = i - n1;
           if (!waited) {
             asm volatile("griddepcontrol.wait;" ::: "memory");
             waited = true;
           }
           const int jx = (j % args.kb2) * kBK;
-          ptx::tma_load_2d_pair(a, &tmA2, bar, jx, row0);
-          ptx::tma_load_2d_pair(b, j < args.kb2 ? &tmB2 : &tmB3, bar, jx, tok0);
+          const int part = j / args.kb2;
+          if (cta == 0) ptx::mbar_arrive_expect_tx(&full[st], 2 * (kABytes + C::kBBytes));
+          ptx::tma_load_2d_pair(a, part < 2 ? &tmA2 : &tmA2u, bar, jx, row0);
+          const CUtensorMap* mB = part == 0 ? &tmB2 : part == 1 ? &tmB3 : part == 2 ? &tmB2u : &tmB3u;
+          ptx::tma_load_2d_pair(b, mB, bar, jx, tok0);
         }
       }
     }
@@ -517,7 +559,7 @@ pair_forward_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_const
     }
   } else if (warp == 1 && lane == 0 && cta == 0) {
     // ---------------------------------------------------------- MMA issuer (even CTA)
-    constexpr uint32_t idesc = ptx::idesc_bf16(2 * kBM, kPairN, 0);
+    constexpr uint32_t idesc = ptx::idesc_bf16(2 * kBM, N, 0);
     bool stop = false;
     int g = 0, j = 0, issued = 0;
     for (int tile = cluster; tile < tiles; tile += n_clusters, ++j) {
@@ -537,15 +579,37 @@ pair_forward_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_const
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t a = ptx::smem_u32(smem + st * kPairStageBytes);
-        const uint32_t b = a + kABytes;
-        // D1 = W0 . X^T over K = I at column 0; D2 = U . (T_hi + T_lo)^T at kPairN
-        const uint32_t d = i < n1 ? tmem : tmem + (uint32_t)kPairN;
-        const bool first = i == 0 || i == n1;
+        const uint32_t a = ptx::smem_u32(smem + st * C::kStageBytes);
+        const uint32_t b = a + C::kNumA * kABytes;
+        if constexpr (MODE == MODE_FORWARD) {
+          // D1 = W0 . X^T over K = I at column 0; D2 = U . (T_hi + T_lo)^T at N
+          const uint32_t d = i < n1 ? tmem : tmem + (uint32_t)N;
+          const bool first = i == 0 || i == n1;
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk)
-          ptx::umma_bf16_pair(d, ptx::sdesc_sw128(a + kk * 32, 16, 1024), ptx::sdesc_sw128(b + kk * 32, 16, 1024),
-                              idesc, (!first || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            ptx::umma_bf16_pair(d, ptx::sdesc_sw128(a + kk * 32, 16, 1024), ptx::sdesc_sw128(b + kk * 32, 16, 1024),
+                                idesc, (!first || kk > 0) ? 1u : 0u);
+        } else if (i < n1) {
+          // D1 of projection q at column q * N, over K = I
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t bd = ptx::sdesc_sw128(b + kk * 32, 16, 1024);
+#pragma unroll
+            for (int q = 0; q < C::kNumA; ++q)
+              ptx::umma_bf16_pair(tmem + (uint32_t)(q * N), ptx::sdesc_sw128(a + q * kABytes + kk * 32, 16, 1024),
+                                  bd, idesc, (i > 0 || kk > 0) ? 1u : 0u);
+          }
+        } else {
+          // D2 of projection q at column (kNumA + q) * N: U . (T_hi + T_lo)^T
+          const int jj = i - n1;
+          const int q = jj / (2 * args.kb2);
+          const int jd = jj % (2 * args.kb2);  // item within its accumulator
+          const uint32_t d2 = tmem + (uint32_t)((C::kNumA + q) * N);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            ptx::umma_bf16_pair(d2, ptx::sdesc_sw128(a + kk * 32, 16, 1024), ptx::sdesc_sw128(b + kk * 32, 16, 1024),
+                                idesc, (jd > 0 || kk > 0) ? 1u : 0u);
+        }
         ptx::umma_commit_pair(&empty[st], kPairMask);
         ++issued;
       }
@@ -560,7 +624,9 @@ pair_forward_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_const
     }
   } else if (warp >= 2) {
     // ---------------------------------------------------------- epilogue (both CTAs)
-    const int quarter = warp & 3;
+    const int quarter = warp & 3;          // a warp reads lanes 32 * (warp % 4) ...
+    const int part = (warp - 2) / 4;       // ... and columns [part * W, (part + 1) * W)
+    constexpr int W = N * 4 / C::kEpiWarps;  // columns per epilogue warp
     const int row = quarter * 32 + lane;  // accumulator row = TMEM lane
     const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
     const bool storer = threadIdx.x == 64;  // issues the TMA stores of the tile
@@ -570,31 +636,53 @@ pair_forward_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_const
     int j = 0;
     for (int tile = cluster; tile < tiles; tile += n_clusters, ++j) {
       const int row0 = (tile / n_tiles) * (2 * kBM) + (int)cta * kBM;
-      const int col0 = (tile % n_tiles) * kPairN;
-      const int ncols = min(kPairN, args.cols - col0);
+      const int col0 = (tile % n_tiles) * N;
+      const int ncols = min(N, args.cols - col0);
       if (storer) ptx::bulk_wait_read();  // the previous tile's store has read sOut
       const bool got = ptx::mbar_wait(accum, (uint32_t)j & 1u, abort_flag);
-      // one decision for all four warps: the barriers below need every one of them
-      ok = ptx::bar_red_and(1, kPairEpi, got);
+      // one decision for all epilogue warps: the barriers below need every one of them
+      ok = ptx::bar_red_and(1, C::kEpi, got);
       if (!ok) break;
       ptx::tc_fence_after();
       const int grow = row0 + row;
       const float so = (grow < args.rows) ? __ldg(args.s + grow) : 0.f;
-      for (int c0 = 0; c0 < ncols; c0 += 16) {
-        float d1[16], d2[16];
-        ptx::tmem_ld16(taddr + c0, d1);
-        if (has_d2) ptx::tmem_ld16(taddr + kPairN + c0, d2);
-        ptx::tmem_wait_ld();
+      float su = 0.f;
+      if constexpr (MODE == MODE_GATE_UP) su = (grow < args.rows) ? __ldg(args.s_up + grow) : 0.f;
+      const int c_begin = C::kEpiWarps == 4 ? 0 : part * W;
+      const int c_end = C::kEpiWarps == 4 ? ncols : min(ncols, (part + 1) * W);
+      for (int c0 = c_begin; c0 < c_end; c0 += 16) {
+        if constexpr (MODE == MODE_GATE_UP) {
+          // gate g = s_g D1g + D2g and up u = s_u D1u + D2u; Y = gelu_tanh(g) u
+          float g1[16], u1[16], g2[16], u2[16];
+          ptx::tmem_ld16(taddr + c0, g1);
+          ptx::tmem_ld16(taddr + N + c0, u1);
+          if (has_d2) {
+            ptx::tmem_ld16(taddr + 2 * N + c0, g2);
+            ptx::tmem_ld16(taddr + 3 * N + c0, u2);
+          }
+          ptx::tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-          sOut[(c0 + e) * kBM + row] = __float2bfloat16_rn(has_d2 ? fmaf(so, d1[e], d2[e]) : so * d1[e]);
+          for (int e = 0; e < 16; ++e) {
+            const float gv = has_d2 ? fmaf(so, g1[e], g2[e]) : so * g1[e];
+            const float uv = has_d2 ? fmaf(su, u1[e], u2[e]) : su * u1[e];
+            sOut[(c0 + e) * kBM + row] = __float2bfloat16_rn(gelu_tanh(gv) * uv);
+          }
+        } else {
+          float d1[16], d2[16];
+          ptx::tmem_ld16(taddr + c0, d1);
+          if (has_d2) ptx::tmem_ld16(taddr + N + c0, d2);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            sOut[(c0 + e) * kBM + row] = __float2bfloat16_rn(has_d2 ? fmaf(so, d1[e], d2[e]) : so * d1[e]);
+        }
       }
       // tensor memory read: the next tile's MMAs may start
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive_cluster(free_bar);
       ptx::fence_proxy_async_smem();
-      asm volatile("bar.sync 1, %0;" ::"n"(kPairEpi) : "memory");
+      asm volatile("bar.sync 1, %0;" ::"n"(C::kEpi) : "memory");
       if (storer) {
         // rows past O and tokens past M fall outside Y and are not written
         ptx::tma_store_2d(&tmY, sOut, row0, col0);
@@ -608,7 +696,7 @@ pair_forward_kernel(const __grid_constant__ CUtensorMap tmA1, const __grid_const
   __syncwarp();
   ptx::tc_fence_before();
   ptx::cluster_sync();  // both epilogues have read their accumulators; every MMA has completed
-  if (warp == 1) ptx::tmem_dealloc_pair(tmem, kPairTmemCols);
+  if (warp == 1) ptx::tmem_dealloc_pair(tmem, C::kTmemCols);
 }
 
 // s (.) W0 for rank 0 (no tensor-core work).
@@ -977,6 +1065,202 @@ recon_band_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constan
   if (warp == 1) ptx::tmem_dealloc(tmem, 2 * kRecN);
 }
 
+// ------------------------------------------------------------- SVD products
+// The randomized SVD's products with a bf16 residual R [O, I] on tensor
+// cores ("The theta bundle" -- Low-rank residual, the randomized algorithm of
+// Halko, Martinsson and Tropp):
+//   R_LEFT   C [O, k] = R . F^T   F [k, I]: the test matrix, or Z^T
+//   !R_LEFT  C [k, I] = F^T . R   F = Q [O, k], given here as Q^T [k, O]
+// F is fp32; it enters as three bf16 parts F = F1 + F2 + F3 (each the
+// rounded remainder of the one before: together the whole 24-bit
+// significand), each multiplied into the same fp32 accumulator, so the sums
+// are of the exact products of the fp32 operands, in another order than a
+// CUDA-core fp32 GEMM. R is bf16, so it enters exactly. K is split over
+// grid z; split z writes its partial C to part + z * M * N (fp32, row-major)
+// and the caller adds the splits in a fixed order.
+// 192 threads as in umma_kernel: TMA warp, MMA warp, four epilogue warps.
+constexpr int kSvdParts = 3;
+
+template <bool R_LEFT>
+struct SvdCfg {
+  static constexpr int kBN = R_LEFT ? 96 : 128;  // N: the samples (k <= 96) / 128 columns of R
+  static constexpr int kNumA = R_LEFT ? 1 : kSvdParts;
+  static constexpr int kNumB = R_LEFT ? kSvdParts : 1;
+  static constexpr int kBBytes = kBN * kBK * 2;
+  static constexpr int kStageBytes = kNumA * kABytes + kNumB * kBBytes;
+  static constexpr int kStages = 3;
+  static constexpr int kTmemCols = 128;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(kStageBytes % 1024 == 0 && kBBytes % 1024 == 0, "swizzled tiles start on 1024-byte boundaries");
+};
+
+struct SvdArgs {
+  int M, N;         // C [M, N]
+  int kb;           // K blocks of 64
+  int splits;       // grid z
+  float* part;      // [splits, M, N]
+  unsigned* err;
+};
+
+// R_LEFT: m0 = R (A, K-major), m1..m3 = the parts of F (B, K-major [k, I]).
+// !R_LEFT: m0..m2 = the parts of Q^T (A, K-major [k, O]), m3 = R (B, MN-major).
+template <bool R_LEFT>
+__global__ void __launch_bounds__(kThreads)
+svd_mma_kernel(const __grid_constant__ CUtensorMap m0, const __grid_constant__ CUtensorMap m1,
+               const __grid_constant__ CUtensorMap m2, const __grid_constant__ CUtensorMap m3, const SvdArgs args) {
+  using C = SvdCfg<R_LEFT>;
+  constexpr int S = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint64_t* empty = full + S;
+  uint64_t* accum = empty + S;
+  uint64_t* drain = accum + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int n_tile = blockIdx.x, m_tile = blockIdx.y, split = blockIdx.z;
+  const int kb_begin = (int)((int64_t)split * args.kb / args.splits);
+  const int kb_end = (int)((int64_t)(split + 1) * args.kb / args.splits);
+  const int total = kb_end - kb_begin;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], 1);
+    }
+    ptx::mbar_init(accum, 1);
+    ptx::mbar_init(drain, 1);
+    *abort_flag = prior_timeout(args.err);
+    ptx::fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, C::kTmemCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+
+  auto give_up = [&]() {
+    record_timeout(args.err);
+    *abort_flag = 1;
+  };
+
+  if (warp == 0 && lane == 0) {
+    // ---------------------------------------------------------- producer
+    int issued = 0;
+    for (int i = 0; i < total; ++i) {
+      const int st = i % S;
+      const uint32_t ph = (uint32_t)(i / S) & 1u;
+      if (!ptx::mbar_wait(&empty[st], ph ^ 1u, abort_flag)) {
+        give_up();
+        break;
+      }
+      uint8_t* a = smem + st * C::kStageBytes;
+      uint8_t* b = a + C::kNumA * kABytes;
+      const int kx = (kb_begin + i) * kBK;
+      ptx::mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+      if constexpr (R_LEFT) {
+        ptx::tma_load_2d(a, &m0, &full[st], kx, m_tile * kBM);
+        ptx::tma_load_2d(b, &m1, &full[st], kx, n_tile * C::kBN);
+        ptx::tma_load_2d(b + C::kBBytes, &m2, &full[st], kx, n_tile * C::kBN);
+        ptx::tma_load_2d(b + 2 * C::kBBytes, &m3, &full[st], kx, n_tile * C::kBN);
+      } else {
+        ptx::tma_load_2d(a, &m0, &full[st], kx, m_tile * kBM);
+        ptx::tma_load_2d(a + kABytes, &m1, &full[st], kx, m_tile * kBM);
+        ptx::tma_load_2d(a + 2 * kABytes, &m2, &full[st], kx, m_tile * kBM);
+        // R [O, I] as the MN-major B: per 64-column atom of N, 64 rows of K (= O)
+#pragma unroll
+        for (int at = 0; at < C::kBN / 64; ++at)
+          ptx::tma_load_2d(b + at * 64 * 128, &m3, &full[st], n_tile * C::kBN + at * 64, kx);
+      }
+      ++issued;
+    }
+    for (int st = 0; st < S && st < issued; ++st) {
+      const int last = st + ((issued - 1 - st) / S) * S;
+      if (!ptx::mbar_wait(&full[st], (uint32_t)(last / S) & 1u, abort_flag)) {
+        int never = 0;
+        ptx::mbar_wait(&full[st], (uint32_t)(last / S) & 1u, &never, 100000000ull);
+      }
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------------------------------------------------- MMA issuer
+    constexpr uint32_t idesc = ptx::idesc_bf16(kBM, C::kBN, R_LEFT ? 0 : 1);
+    int done = 0;
+    for (int i = 0; i < total; ++i) {
+      const int st = i % S;
+      const uint32_t ph = (uint32_t)(i / S) & 1u;
+      if (!ptx::mbar_wait(&full[st], ph, abort_flag)) {
+        give_up();
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t a = ptx::smem_u32(smem + st * C::kStageBytes);
+      const uint32_t b = a + C::kNumA * kABytes;
+#pragma unroll
+      for (int kk = 0; kk < kBK / 16; ++kk) {
+#pragma unroll
+        for (int p = 0; p < kSvdParts; ++p) {
+          const uint64_t ad = R_LEFT ? ptx::sdesc_sw128(a + kk * 32, 16, 1024)
+                                     : ptx::sdesc_sw128(a + p * kABytes + kk * 32, 16, 1024);
+          const uint64_t bd = R_LEFT ? ptx::sdesc_sw128(b + p * C::kBBytes + kk * 32, 16, 1024)
+                                     : ptx::sdesc_sw128(b + kk * 16 * 128, 64 * 128, 1024);
+          ptx::umma_bf16(tmem, ad, bd, idesc, (i > 0 || kk > 0 || p > 0) ? 1u : 0u);
+        }
+      }
+      ptx::umma_commit(&empty[st]);
+      ++done;
+    }
+    if (done == total) {
+      ptx::umma_commit(accum);
+    } else if (done > 0) {
+      ptx::umma_commit(drain);
+      int never = 0;
+      ptx::mbar_wait(drain, 0, &never);
+    }
+  } else if (warp >= 2) {
+    // ---------------------------------------------------------- epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16);
+    // an empty split (more splits than K blocks) leaves a zero partial
+    bool ok = total == 0 || ptx::mbar_wait(accum, 0, abort_flag);
+    if (!ok) give_up();
+    ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
+    ptx::tc_fence_after();
+    const int m = m_tile * kBM + row;
+    const int n0 = n_tile * C::kBN;
+    const int ncols = min(C::kBN, args.N - n0);
+    float* out = args.part + (int64_t)split * args.M * args.N + (int64_t)m * args.N + n0;
+    if (ok) {
+      for (int c0 = 0; c0 < ncols; c0 += 16) {
+        float d[16];
+        if (total > 0) {
+          ptx::tmem_ld16(taddr + c0, d);
+          ptx::tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) d[e] = 0.f;
+        }
+        if (m < args.M) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            if (c0 + e < ncols) out[c0 + e] = d[e];
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) ptx::tmem_dealloc(tmem, C::kTmemCols);
+}
+
 // ------------------------------------------------------------------ host side
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -1135,22 +1419,28 @@ cudaError_t launch_tile_kernel(const LaunchCtx& c, const Maps& mp, Args args, in
                     c.stream, args.splits, mp.a1, mp.b1, mp.a2, mp.b2, mp.b3, mp.a1u, mp.a2u, mp.b2u, mp.b3u, args);
 }
 
-// The persistent CTA-pair forward: one cluster of two per pair of SMs that
+// The persistent CTA-pair kernel: one cluster of two per pair of SMs that
 // can hold one (the occupancy query, once per device), at most one per tile.
-cudaError_t launch_pair_forward(const LaunchCtx& c, const Maps& mp, const CUtensorMap& mY, const Args& args,
-                                int64_t tiles) {
-  auto kern = pair_forward_kernel;
+// Y [M, O] is written by TMA in boxes of 128 rows of W0 (columns of Y) x one
+// tile's tokens.
+template <int MODE>
+cudaError_t launch_pair(const LaunchCtx& c, const Maps& mp, const Args& args, void* Y, cudaError_t* ce_map) {
+  using C = PairCfg<MODE>;
+  auto kern = pair_kernel<MODE>;
   static KernelInfo info[64];
   static int max_clusters[64];
-  cudaError_t e = prepare_kernel(&info[c.device], c.device, kern, kThreads, kPairSmemBytes, kPairTmemCols, false);
+  CUtensorMap mY;
+  if (make_map_box(&mY, Y, args.cols, args.rows, C::kN, kBM, CU_TENSOR_MAP_SWIZZLE_NONE, ce_map))
+    return *ce_map;
+  cudaError_t e = prepare_kernel(&info[c.device], c.device, kern, C::kThreads, C::kSmemBytes, C::kTmemCols, false);
   if (e != cudaSuccess) return e;
   {
     std::lock_guard<std::mutex> lk(setup_mutex());
     if (max_clusters[c.device] == 0) {
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(2, 1, 1);
-      cfg.blockDim = dim3(kThreads, 1, 1);
-      cfg.dynamicSmemBytes = kPairSmemBytes;
+      cfg.blockDim = dim3(C::kThreads, 1, 1);
+      cfg.dynamicSmemBytes = C::kSmemBytes;
       cudaLaunchAttribute attr;
       attr.id = cudaLaunchAttributeClusterDimension;
       attr.val.clusterDim.x = 2;
@@ -1167,9 +1457,10 @@ cudaError_t launch_pair_forward(const LaunchCtx& c, const Maps& mp, const CUtens
       max_clusters[c.device] = n;
     }
   }
+  const int64_t tiles = ceil_div(args.rows, 2 * kBM) * ceil_div(args.cols, C::kN);
   const int64_t clusters = tiles < max_clusters[c.device] ? tiles : max_clusters[c.device];
-  return launch_pdl(kern, dim3((unsigned)(2 * clusters), 1, 1), dim3(kThreads), kPairSmemBytes, c.stream, 2, mp.a1,
-                    mp.b1, mp.a2, mp.b2, mp.b3, mY, args);
+  return launch_pdl(kern, dim3((unsigned)(2 * clusters), 1, 1), dim3(C::kThreads), C::kSmemBytes, c.stream, 2, mp.a1,
+                    mp.b1, mp.a2, mp.b2, mp.b3, mp.a1u, mp.a2u, mp.b2u, mp.b3u, mY, args);
 }
 
 template <int KB>
@@ -1292,7 +1583,7 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
   // CTA gets a whole tile -- under the throughput policy, or when the tiles
   // already fill the GPU (the latency policy would not split K then either).
   const bool pair = BN == 256 && (c.policy == THETA_POLICY_THROUGHPUT || (int64_t)m_tiles * n_tiles >= c.num_sms);
-  const int box_b = pair ? kPairHalf : BN;  // tokens per B box
+  const int box_b = pair ? PairCfg<MODE_FORWARD>::kHalf : BN;  // tokens per B box
   Maps mp;
   if ((st = make_map(&mp.a1, W0, O, I, kBM, ce))) return st;
   if ((st = make_map(&mp.b1, X, M, I, box_b, ce))) return st;
@@ -1317,10 +1608,7 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
   a.err = c.err;
   if (pair) {
     a.splits = 1;
-    // Y [M, O] written by TMA: boxes of 128 rows of W0 (columns of Y) x 256 tokens
-    CUtensorMap mY;
-    if ((st = make_map_box(&mY, Y, M, O, kPairN, kBM, CU_TENSOR_MAP_SWIZZLE_NONE, ce))) return st;
-    e = launch_pair_forward(c, mp, mY, a, ceil_div(O, 2 * kBM) * ceil_div(M, kPairN));
+    e = launch_pair<MODE_FORWARD>(c, mp, a, Y, ce);
     if (e != cudaSuccess) {
       *ce = e;
       return THETA_ERR_CUDA;
@@ -1366,17 +1654,21 @@ int launch_gate_up_umma(const LaunchCtx& c, const void* X, const void* W0g, cons
   const int BN = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
   const int m_tiles = (int)ceil_div(O, kBM);
   const int n_tiles = (int)ceil_div(M, BN);
+  // More than 256 tokens: CTA pairs share 256-row x 128-token tiles, on the
+  // same condition as the forward's pairs
+  const bool pair = M > 256 && (c.policy == THETA_POLICY_THROUGHPUT || (int64_t)m_tiles * n_tiles >= c.num_sms);
+  const int box_b = pair ? PairCfg<MODE_GATE_UP>::kHalf : BN;  // tokens per B box
   Maps mp;
   if ((st = make_map(&mp.a1, W0g, O, I, kBM, ce))) return st;
   if ((st = make_map(&mp.a1u, W0u, O, I, kBM, ce))) return st;
-  if ((st = make_map(&mp.b1, X, M, I, BN, ce))) return st;
+  if ((st = make_map(&mp.b1, X, M, I, box_b, ce))) return st;
   if (r > 0) {
     if ((st = make_map(&mp.a2, Ug, O, r, kBM, ce))) return st;
-    if ((st = make_map(&mp.b2, t[0], M, r, BN, ce))) return st;
-    if ((st = make_map(&mp.b3, t[1], M, r, BN, ce))) return st;
+    if ((st = make_map(&mp.b2, t[0], M, r, box_b, ce))) return st;
+    if ((st = make_map(&mp.b3, t[1], M, r, box_b, ce))) return st;
     if ((st = make_map(&mp.a2u, Uu, O, r, kBM, ce))) return st;
-    if ((st = make_map(&mp.b2u, t[2], M, r, BN, ce))) return st;
-    if ((st = make_map(&mp.b3u, t[3], M, r, BN, ce))) return st;
+    if ((st = make_map(&mp.b2u, t[2], M, r, box_b, ce))) return st;
+    if ((st = make_map(&mp.b3u, t[3], M, r, box_b, ce))) return st;
   } else {
     mp.a2 = mp.a2u = mp.a1;
     mp.b2 = mp.b3 = mp.b2u = mp.b3u = mp.b1;
@@ -1392,6 +1684,15 @@ int launch_gate_up_umma(const LaunchCtx& c, const void* X, const void* W0g, cons
   a.early_start = r > 0;  // directly after the up projection's T = X.V kernel
   a.err = c.err;
   cudaError_t e;
+  if (pair) {
+    a.splits = 1;
+    e = launch_pair<MODE_GATE_UP>(c, mp, a, Y, ce);
+    if (e != cudaSuccess) {
+      *ce = e;
+      return THETA_ERR_CUDA;
+    }
+    return THETA_OK;
+  }
   switch (BN) {
     case 16: e = launch_tile_kernel<16, MODE_GATE_UP>(c, mp, a, m_tiles, n_tiles); break;
     case 32: e = launch_tile_kernel<32, MODE_GATE_UP>(c, mp, a, m_tiles, n_tiles); break;
@@ -1470,6 +1771,87 @@ int launch_reconstruct_umma(const LaunchCtx& c, const float* s, const void* W0, 
     case 3: e = launch_recon<3>(c, mU, mV, mW0, mOut, s, (int)O, (int)I); break;
     default: e = launch_recon<4>(c, mU, mV, mW0, mOut, s, (int)O, (int)I); break;
   }
+  if (e != cudaSuccess) {
+    *ce = e;
+    return THETA_ERR_CUDA;
+  }
+  return THETA_OK;
+}
+
+namespace {
+
+template <bool R_LEFT>
+cudaError_t launch_svd_mma_t(const LaunchCtx& c, const CUtensorMap* maps, const SvdArgs& a, int m_tiles,
+                             int n_tiles) {
+  using C = SvdCfg<R_LEFT>;
+  auto kern = svd_mma_kernel<R_LEFT>;
+  static KernelInfo info[64];
+  cudaError_t e = prepare_kernel(&info[c.device], c.device, kern, kThreads, C::kSmemBytes, C::kTmemCols, false);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(kern, dim3((unsigned)n_tiles, (unsigned)m_tiles, (unsigned)a.splits), dim3(kThreads),
+                    C::kSmemBytes, c.stream, 1, maps[0], maps[1], maps[2], maps[3], a);
+}
+
+}  // namespace
+
+int svd_mma_splits(const LaunchCtx& c, bool r_left, int64_t O, int64_t I, int k) {
+  const int64_t tiles = r_left ? ceil_div(O, kBM) : ceil_div(I, SvdCfg<false>::kBN) * ceil_div(k, kBM);
+  const int64_t kb = ceil_div(r_left ? I : O, kBK);
+  // one CTA per SM; the split count that finishes the K blocks in the fewest
+  // rounds of CTAs, each split keeping at least four K blocks
+  int best = 1;
+  int64_t best_cost = -1;
+  for (int sp = 1; sp <= kSvdMaxSplits; ++sp) {
+    if (sp > 1 && kb / sp < 4) break;
+    const int64_t cost = ceil_div(tiles * sp, (int64_t)c.num_sms) * ceil_div(kb, (int64_t)sp);
+    if (best_cost < 0 || cost < best_cost) best = sp, best_cost = cost;
+  }
+  return best;
+}
+
+int launch_svd_mma(const LaunchCtx& c, bool r_left, const void* R, int64_t O, int64_t I, const void* parts,
+                   int64_t part_stride, int64_t part_pitch, int k, int splits, float* part_out, cudaError_t* ce) {
+  *ce = cudaSuccess;
+  CUtensorMap maps[4];
+  int st;
+  const bf16* P = static_cast<const bf16*>(parts);
+  const int64_t part_elems = part_stride;
+  SvdArgs a = {};
+  a.splits = splits;
+  a.part = part_out;
+  a.err = c.err;
+  if (r_left) {
+    // C [O, k] = R . F^T: R rows by 128, the k samples as one N tile
+    if ((st = make_map_box(&maps[0], R, O, I, kBM, kBK, CU_TENSOR_MAP_SWIZZLE_128B, ce))) return st;
+    for (int p = 0; p < kSvdParts; ++p)
+      if ((st = make_map_box(&maps[1 + p], P + p * part_elems, k, I, SvdCfg<true>::kBN, kBK,
+                             CU_TENSOR_MAP_SWIZZLE_128B, ce)))
+        return st;
+    a.M = (int)O, a.N = k, a.kb = (int)ceil_div(I, kBK);
+  } else {
+    // C [k, I] = Q^T . R: the parts of Q^T [k, O] (row pitch part_pitch) as A,
+    // R as the MN-major B in boxes of 64 columns x 64 rows
+    for (int p = 0; p < kSvdParts; ++p) {
+      EncodeTiledFn enc = encode_fn(ce);
+      if (!enc) return THETA_ERR_CUDA;
+      cuuint64_t dims[2] = {(cuuint64_t)O, (cuuint64_t)k};
+      cuuint64_t strides[1] = {(cuuint64_t)part_pitch * 2};
+      cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kBM};
+      cuuint32_t estr[2] = {1, 1};
+      if (enc(&maps[p], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<bf16*>(P + p * part_elems), dims, strides,
+              box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+        *ce = cudaErrorInvalidValue;
+        return THETA_ERR_CUDA;
+      }
+    }
+    if ((st = make_map_box(&maps[3], R, O, I, kBK, 64, CU_TENSOR_MAP_SWIZZLE_128B, ce))) return st;
+    a.M = k, a.N = (int)I, a.kb = (int)ceil_div(O, kBK);
+  }
+  const int m_tiles = (int)ceil_div(a.M, kBM);
+  const int n_tiles = (int)ceil_div(a.N, r_left ? SvdCfg<true>::kBN : SvdCfg<false>::kBN);
+  const cudaError_t e = r_left ? launch_svd_mma_t<true>(c, maps, a, m_tiles, n_tiles)
+                               : launch_svd_mma_t<false>(c, maps, a, m_tiles, n_tiles);
   if (e != cudaSuccess) {
     *ce = e;
     return THETA_ERR_CUDA;

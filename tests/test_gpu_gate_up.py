@@ -53,6 +53,13 @@ CASES = [
     (64, 1024, 1152, 0),     # rank 0
     (3, 1024, 6912, 16),     # deep K: split across a cluster
     (128, 392, 1160, 256),   # maximum rank
+    # more than 256 tokens: under the throughput policy CTA pairs share
+    # 256-row x 128-token tiles (ragged rows past O, tokens past M, K not a
+    # multiple of 64, rank 0, the largest rank)
+    (257, 264, 392, 40),
+    (600, 392, 1160, 256),
+    (520, 1032, 264, 0),
+    (1100, 520, 1096, 16),
 ]
 
 

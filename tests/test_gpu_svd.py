@@ -67,6 +67,24 @@ def test_matches_oracle_on_a_decaying_spectrum(lib, torch, O, I, r, k, power_ite
     assert np.allclose(nrm, np.linalg.norm(Uo, axis=0), rtol=1e-4, atol=1e-6 * scale)
 
 
+@pytest.mark.parametrize("power_iters", [0, 2])
+@pytest.mark.parametrize("O,I,r,k", [(1152, 6912, 32, 42), (300, 200, 8, 14), (513, 264, 1, 4), (264, 392, 40, 40),
+                                     (2056, 1160, 64, 74)])
+def test_bf16_residual_matches_oracle(lib, torch, O, I, r, k, power_iters):
+    """A bf16 residual (I a multiple of 8): the products with R run on tensor
+    cores, the fp32 factor in three bf16 parts. Against the oracle on the
+    same stored R; U and V come back in bf16, so the bound is bf16's."""
+    R, sig = decaying(O, I, min(O, I), 0.8, O * 5 + I)
+    R = oracle.round_to(R * 0.02, "bf16")
+    omega = np.random.default_rng(r + k + 1).standard_normal((k, I))
+    U, V = gpu_svd(lib, torch, R, r, omega, power_iters, "bf16")
+    Uo, Vo = oracle.randomized_svd(R, r, omega, power_iters)
+    scale = np.linalg.norm(Uo @ Vo.T)
+    assert np.linalg.norm(U @ V.T - Uo @ Vo.T) <= 1e-2 * scale
+    nrm, nrm_o = np.linalg.norm(U, axis=0), np.linalg.norm(Uo, axis=0)
+    assert np.allclose(nrm, nrm_o, rtol=1e-2, atol=1e-3 * nrm_o[0])
+
+
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
 def test_flat_spectrum_residual_error_matches_oracle(lib, torch, dt):
     """The pages' kind of residual (no spectral knee): a Gemma-3-1B gate layer
