@@ -1107,6 +1107,17 @@ def run_op(args):
         out = torch.empty(O, I, dtype=torch.bfloat16, device="cuda")
         call = lambda: theta.theta_reconstruct(s, W0, U, V, out)  # noqa: E731
         nbytes, nflops = bytes_reconstruct(O, I, r), 2 * O * I * r
+    elif args.op == "reconstruct_band":
+        # the --layers layers of one band: one shared W0, each layer's s, U, V
+        W0 = syn.device_normal((O, I), 0.02, seed, "W0", O, I)
+        sl = [1.0 + syn.device_normal((O,), 0.05, seed + l, "s", O, dtype="f32") for l in range(L)]
+        Ul = [syn.device_normal((O, r), 0.01, seed + l, "U", O, r) for l in range(L)] if r else None
+        Vl = [syn.device_normal((I, r), 0.01, seed + l, "V", I, r) for l in range(L)] if r else None
+        outs = [torch.empty(O, I, dtype=torch.bfloat16, device="cuda") for _ in range(L)]
+        call = lambda: theta.theta_reconstruct_band(sl, W0, Ul, Vl, outs)  # noqa: E731
+        # W0 read once for the band; every layer's s, U, V read and W written
+        nbytes = O * I * BF16 + L * (bytes_reconstruct(O, I, r) - O * I * BF16)
+        nflops = L * 2 * O * I * r
     elif args.op == "prelude":
         W = syn.device_family_weights(L, O, I, seed=seed, family="op")
         W0 = [torch.empty(O, I, dtype=torch.bfloat16, device="cuda") for _ in range(G)]
@@ -1198,7 +1209,7 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-rows", type=int, default=8)
     ap.add_argument("--op", choices=["forward", "layer_forward", "forward_nvfp4", "gate_up", "grouped", "reconstruct",
-                                     "prelude", "frob", "svd"],
+                                     "reconstruct_band", "prelude", "frob", "svd"],
                     help="time one entry point on one problem instead of the whole step")
     ap.add_argument("--model", choices=["1b", "31b"], default="31b", help="--op layer_forward: the model's shapes")
     ap.add_argument("--policy", choices=["latency", "throughput"], default="latency",

@@ -1018,16 +1018,28 @@ recon_band_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constan
     // tcgen05.ld is warp-collective. A wait can succeed in one warp and give
     // up in another when an abort lands just as the barrier completes.
     bool ok = ptx::bar_red_and(1, kBandEpi, ptx::mbar_wait(w_full, 0, abort_flag));
+    // this thread's 64 W0 values, unpacked once for all the band's layers
+    const uint8_t* wbox = sW + half * kABytes + row * 128;
+    float w0f[64];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int chunk = k ^ (row & 7);  // 128-byte swizzle of 16-byte chunks
+      unpack(*reinterpret_cast<const uint4*>(wbox + chunk * 16), *reinterpret_cast<float(*)[8]>(w0f + 8 * k));
+    }
+    // each layer's row scale is loaded one layer ahead, off the critical path
+    const bool in_rows = o0 + row < a.O;
+    float s_next = (n > 0 && in_rows) ? __ldg(a.s[0] + o0 + row) : 0.f;
     for (int l = 0; l < n && ok; ++l) {
       const int b = l & 1;
       const uint32_t taddr = taddr0 + (uint32_t)(b * kRecN);
+      const float so = s_next;
+      if (l + 1 < n) s_next = in_rows ? __ldg(a.s[l + 1] + o0 + row) : 0.f;
       const bool got = ptx::mbar_wait(&acc_full[b], (uint32_t)((l >> 1) & 1), abort_flag);
       // the store of layer l - kOutBufs read its buffer before this layer rewrites it
       if (leader) ptx::bulk_wait_read_n<C::kOutBufs - 1>();
       ok = ptx::bar_red_and(1, kBandEpi, got);
       if (!ok) break;
       ptx::tc_fence_after();
-      const float so = (o0 + row < a.O) ? __ldg(a.s[l] + o0 + row) : 0.f;
       // this warp's 64 columns (one swizzled box of the tile): all four loads
       // in flight, one wait
       float d[64];
@@ -1036,15 +1048,13 @@ recon_band_kernel(const __grid_constant__ CUtensorMap tmW0, const __grid_constan
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
       ptx::mbar_arrive(&acc_free[b]);  // tensor memory read: layer l+2's MMAs may start
-      const uint8_t* wbox = sW + half * kABytes + row * 128;
       uint8_t* obox = sOut + (l % C::kOutBufs) * C::kTileBytes + half * kABytes + row * 128;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const int chunk = k ^ (row & 7);  // 128-byte swizzle of 16-byte chunks
-        float w[8], o[8];
-        unpack(*reinterpret_cast<const uint4*>(wbox + chunk * 16), w);
+        const int chunk = k ^ (row & 7);
+        float o[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = fmaf(so, w[e], d[8 * k + e]);
+        for (int e = 0; e < 8; ++e) o[e] = fmaf(so, w0f[8 * k + e], d[8 * k + e]);
         *reinterpret_cast<uint4*>(obox + chunk * 16) = pack(o, (uint4*)nullptr);
       }
       ptx::fence_proxy_async_smem();
