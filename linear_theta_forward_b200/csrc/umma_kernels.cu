@@ -801,8 +801,10 @@ recon_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
     }
   }
 
-  // epilogue: warp w owns tensor-memory lanes (rows) 32w .. 32w+31
+  // epilogue: warp w owns tensor-memory lanes (rows) 32w .. 32w+31; the row
+  // scale is loaded before the waits, off the critical path
   const int row = warp * 32 + lane;
+  const float so = (o0 + row < O) ? __ldg(s + o0 + row) : 0.f;
   bool ok = ptx::mbar_wait(bar_acc, 0, abort_flag) && ptx::mbar_wait(bar_w, 0, abort_flag);
   if (!ok && !*abort_flag) {
     record_timeout(err);
@@ -810,23 +812,26 @@ recon_kernel(const __grid_constant__ CUtensorMap tmU, const __grid_constant__ CU
   }
   ok = __all_sync(0xffffffffu, ok);  // tcgen05.ld below is warp-collective
   ptx::tc_fence_after();
-  const float so = (o0 + row < O) ? __ldg(s + o0 + row) : 0.f;
   const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
   if (ok) {
+    // one 64-column box of the tile at a time: four tensor-memory loads in
+    // flight, one wait
 #pragma unroll 1
-    for (int c0 = 0; c0 < kRecN; c0 += 16) {
-      float d[16];
-      ptx::tmem_ld16(taddr + c0, d);
-      ptx::tmem_wait_ld();
-      uint8_t* rowp = sW + (c0 / kBK) * kABytes + row * 128;
+    for (int bx = 0; bx < kRecN / kBK; ++bx) {
+      float d[kBK];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int chunk = ((c0 % kBK) / 8 + h) ^ (row & 7);  // 128-byte swizzle of 16-byte chunks
+      for (int q = 0; q < kBK / 16; ++q)
+        ptx::tmem_ld16(taddr + bx * kBK + q * 16, *reinterpret_cast<float(*)[16]>(d + 16 * q));
+      ptx::tmem_wait_ld();
+      uint8_t* rowp = sW + bx * kABytes + row * 128;
+#pragma unroll
+      for (int k = 0; k < kBK / 8; ++k) {
+        const int chunk = k ^ (row & 7);  // 128-byte swizzle of 16-byte chunks
         uint4* p = reinterpret_cast<uint4*>(rowp + chunk * 16);
         float w[8], o[8];
         unpack(*p, w);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) o[e] = fmaf(so, w[e], d[8 * h + e]);
+        for (int e = 0; e < 8; ++e) o[e] = fmaf(so, w[e], d[8 * k + e]);
         *p = pack(o, (uint4*)nullptr);
       }
     }
