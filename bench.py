@@ -277,7 +277,7 @@ KERNEL_NAMES = {
     "reconstruct": "recon_kernel",
     "frob": "frob_partial_kernel + frob_final_kernel",
     "forward_decode": "gemv_rows_kernel / grouped_rows_kernel / umma_kernel<16..64,FORWARD>",
-    "forward_ridge": "umma_kernel<128,FORWARD> (+ umma_kernel<64,XV>)",
+    "forward_ridge": "pair_kernel<FORWARD> (+ umma_kernel<64,XV>)",
     "forward_prefill": "pair_kernel<FORWARD> (+ umma_kernel<64,XV>)",
 }
 

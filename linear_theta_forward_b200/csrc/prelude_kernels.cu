@@ -491,14 +491,14 @@ prelude_band2_kernel(const __grid_constant__ PreludeArgs a) {
 
 // Threads per output row (32..256, i.e. 8..1 rows per item): the fewest
 // that keep each thread at <= 12 vectors of a row and an item's shared
-// memory within 32 KB, so a CTA has several items in flight and each item
-// carries enough bytes to pay for its one reduction barrier. Vectors per
-// thread are rounded up to a compiled variant.
-bool geometry(int64_t nv, int64_t per_row_bytes, int* tpr, int* vpt) {
+// memory within item_cap, so a CTA has several items in flight and each
+// item carries enough bytes to pay for its one reduction barrier. Vectors
+// per thread are rounded up to a compiled variant.
+bool geometry(int64_t nv, int64_t per_row_bytes, int64_t item_cap, int* tpr, int* vpt) {
   const int tprs[] = {32, 64, 128, 256};
   *tpr = 0;
   for (int c : tprs) {
-    if (ceil_div(nv, c) <= 12 && (kConsumers / c) * per_row_bytes <= 32 * 1024) {
+    if (ceil_div(nv, c) <= 12 && (kConsumers / c) * per_row_bytes <= item_cap) {
       *tpr = c;
       break;
     }
@@ -557,7 +557,12 @@ bool plan(const LaunchCtx& c, const void* const* w, int L, int G, const int32_t*
   if (BAND && nmax > 4) return false;
   const int64_t row_bytes = I * (int64_t)sizeof(T);
   const int64_t per_row = BAND ? nmax * row_bytes : 2 * row_bytes;
-  if (!geometry(I / Vec<T>::N, per_row, tpr, vpt)) return false;
+  // Items of up to 32 KB; the row mode takes up to 48 KB: at the 31B width
+  // that is two rows per item with 128 threads each instead of one with 256,
+  // measured 12% faster (its consumers are issue-bound, and two rows share
+  // one reduction barrier). A larger cap would give BAND mode variants whose
+  // registers keep two CTAs off an SM.
+  if (!geometry(I / Vec<T>::N, per_row, BAND ? 32 * 1024 : 48 * 1024, tpr, vpt)) return false;
   const int rows = kConsumers / *tpr;
   const int64_t slot = ceil_div(rows * per_row, 128) * 128;
   int64_t slots = kSmemBudget / slot;

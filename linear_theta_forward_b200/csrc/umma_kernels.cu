@@ -1597,7 +1597,11 @@ int launch_forward_umma(const LaunchCtx& c, const void* X, const void* W0, const
   // More than 256 tokens: pairs of SMs share 256 x 256 tiles whenever every
   // CTA gets a whole tile -- under the throughput policy, or when the tiles
   // already fill the GPU (the latency policy would not split K then either).
-  const bool pair = BN == 256 && (c.policy == THETA_POLICY_THROUGHPUT || (int64_t)m_tiles * n_tiles >= c.num_sms);
+  // 129 to 256 tokens under the throughput policy: one 256-token pair tile
+  // per 256 rows instead of two 128-token one-SM tiles (measured 5-8% faster
+  // on a stream of Gemma-3-1B-shaped calls).
+  const bool pair = (BN == 256 && (c.policy == THETA_POLICY_THROUGHPUT || (int64_t)m_tiles * n_tiles >= c.num_sms)) ||
+                    (BN == 128 && M > 128 && c.policy == THETA_POLICY_THROUGHPUT);
   const int box_b = pair ? PairCfg<MODE_FORWARD>::kHalf : BN;  // tokens per B box
   Maps mp;
   if ((st = make_map(&mp.a1, W0, O, I, kBM, ce))) return st;

@@ -125,6 +125,9 @@ PAIR_CASES = [
     (520, 1032, 264, 0),     # rank 0: no D2
     (300, 264, 392, 256),    # four rank blocks, hi and lo parts each
     (2100, 520, 1096, 16),
+    (200, 264, 1160, 40),    # 129-256 tokens: one pair tile, the odd CTA's tokens partly past M
+    (256, 1152, 1024, 32),
+    (129, 392, 328, 8),
 ]
 
 
