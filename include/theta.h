@@ -169,12 +169,17 @@ int theta_decompose_prelude(const void* const* weights, int num_layers, int G, i
  *   R [O, I] (dt); omega fp32 [samples, I], the Gaussian test matrix (the
  *   caller draws it; samples = rank + oversampling); U [O, rank] and
  *   V [I, rank] (dt), written. 1 <= rank <= samples <= min(96, O, I);
- *   0 <= power_iters <= 8.
+ *   0 <= power_iters <= 8; O, I <= 4,194,240 (larger: THETA_ERR_UNSUPPORTED).
  *   workspace  device scratch of theta_workspace_size(THETA_OP_RESIDUAL_SVD,
  *              samples, O, I, rank, dt) bytes (M carries samples).
- * fp32 arithmetic on CUDA cores (fp64 for the k x k steps): decomposition
- * work, not the projection's hot path. A direction the sample lacks (R of
- * rank below samples) comes out as a zero column of U and V.
+ * fp32 arithmetic (fp64 for the k x k steps): decomposition work, not the
+ * projection's hot path. For a bf16 R with I a multiple of 8 and R 16-byte
+ * aligned, the products that stream R (R . omega^T, Q^T . R, R . Z) run on
+ * tensor cores with the fp32 factor split exactly into three bf16 parts
+ * (sums of the exact products of the fp32 operands, in another order than
+ * an fp32 GEMM); every other product, and every product of an fp32 R, runs
+ * on CUDA cores. A direction the sample lacks (R of rank below samples)
+ * comes out as a zero column of U and V.
  */
 int theta_residual_svd(const void* R, int64_t O, int64_t I, theta_dtype dt, int rank, int samples,
                        int power_iters, const float* omega, void* U, void* V, void* workspace,

@@ -476,6 +476,9 @@ THETA_API int theta_residual_svd(const void* R, int64_t O, int64_t I, theta_dtyp
                 "theta_residual_svd: need O, I >= 1, 1 <= rank <= samples and 0 <= power_iters <= 8");
   if (samples > svd_max_samples() || samples > O || samples > I)
     return fail(THETA_ERR_UNSUPPORTED, "theta_residual_svd: samples must be <= min(%d, O, I)", svd_max_samples());
+  // the products' grids tile O and I by 64 along grid y (at most 65535)
+  if (O > kSimtMaxRows || I > kSimtMaxRows)
+    return fail(THETA_ERR_UNSUPPORTED, "theta_residual_svd: O and I must be <= %lld", (long long)kSimtMaxRows);
   if (!R || !omega || !U || !V) return fail(THETA_ERR_INVALID_ARG, "theta_residual_svd: NULL pointer");
   const size_t need = svd_workspace_bytes(O, I, samples, rank);
   if (!workspace || workspace_bytes < need || !aligned16(workspace))

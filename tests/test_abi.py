@@ -197,6 +197,9 @@ def test_residual_svd_validation(lib):
     assert raw.theta_residual_svd(p, 200, 200, 0, 4, 97, 1, p, p, p, p, 1 << 30, None) == -2  # samples > 96
     assert raw.theta_residual_svd(p, 64, 20, 0, 4, 24, 1, p, p, p, p, 1 << 30, None) == -2    # samples > I
     assert raw.theta_residual_svd(p, 64, 64, 0, 4, 8, 1, p, p, p, None, 0, None) == -6        # no workspace
+    big_rows = 65535 * 64 + 1  # past the products' grid limit: refused on the host
+    assert raw.theta_residual_svd(p, big_rows, 64, 0, 4, 8, 1, p, p, p, p, 1 << 62, None) == -2
+    assert raw.theta_residual_svd(p, 64, big_rows, 0, 4, 8, 1, p, p, p, p, 1 << 62, None) == -2
     small = lib.theta_workspace_size(lib.THETA_OP_RESIDUAL_SVD, 8, 64, 64, 4, lib.THETA_F32)
     big = lib.theta_workspace_size(lib.THETA_OP_RESIDUAL_SVD, 74, 21504, 5376, 64, lib.THETA_BF16)
     assert small >= 4 * (2 * 64 * 8 + 3 * 8 * 64) and big > small
